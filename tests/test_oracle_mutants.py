@@ -1,0 +1,127 @@
+"""Planted-mistake check for the oracle pins.
+
+Each case copies oracle.c, plants one plausible mistake (wrong chunk index, a
+dropped diagonal, a wrong sign, a transposed operand, a wrong GQA map, a dropped
+scale ...), builds it on the CPU into a temporary directory and runs the pin
+checks against it: every mutant must fail at least one of them.  Nothing here
+touches a GPU or the product library.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import brute
+from sequence_sharded_causal_b200 import inputs
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "second_chunk_index": ("(int64_t)(2 * D - 1 - r) * C", "(int64_t)(2 * D - 2 - r) * C"),
+    "chunks_swapped": ("if (j < C)\n        return (int64_t)r * C + j;",
+                       "if (j >= C)\n        return (int64_t)r * C + (j - C);"),
+    "diagonal_dropped": ("causal ? p + 1 : S", "causal ? (p > 0 ? p : 1) : S"),
+    "lse_sign": ("double lse = m + log(l);", "double lse = m - log(l);"),
+    "gqa_modulo": ("v, b, h / G, s_buf, o + (row * Hq + h) * d, &nk);",
+                   "v, b, h % Hkv, s_buf, o + (row * Hq + h) * d, &nk);"),
+    "scale_dropped_fwd": ("s_buf[key] = scale * dot;", "s_buf[key] = dot;"),
+    "dk_scale_dropped": ("dk[kofs + t] += scale * ds_buf[key] * q_row[t];",
+                         "dk[kofs + t] += ds_buf[key] * q_row[t];"),
+    "ds_sign": ("ds_buf[key] = p_buf[key] * (dp - dlt);", "ds_buf[key] = p_buf[key] * (dlt - dp);"),
+    "dq_uses_v": ("dq_row[t] += scale * ds_buf[key] * k[kofs + t];",
+                  "dq_row[t] += scale * ds_buf[key] * v[kofs + t];"),
+    "dv_uses_ds": ("dv[kofs + t] += p_buf[key] * do_row[t];",
+                   "dv[kofs + t] += ds_buf[key] * do_row[t];"),
+    "delta_dropped": ("dlt += do_row[t] * o_row[t];", "dlt += 0.0 * o_row[t];"),
+    "kend_off_by_one": ("return largest / bk + 1;", "return largest / bk;"),
+    "order_ascending": ("return a->key_work > b->key_work ? -1 : 1;",
+                        "return a->key_work < b->key_work ? -1 : 1;"),
+}
+
+
+def _build_mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / f"lib{name}.so"
+    subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", str(path), "-o",
+                    str(lib), "-lm"], check=True)
+    return str(lib)
+
+
+def _pins_pass():
+    """A compact subset of the pin suite; returns False at the first failure."""
+    rng = np.random.default_rng(1)
+    # zigzag balance + bijection
+    for S, D in ((16, 2), (48, 3), (64, 4)):
+        perm, _ = oracle.partition(S, D)
+        if not np.array_equal(np.sort(perm), np.arange(S)):
+            return False
+        C, twoC = S // (2 * D), S // D
+        pairs = {int((perm[r * twoC:(r + 1) * twoC].astype(np.int64) + 1).sum()) for r in range(D)}
+        if pairs != {C * C * (2 * D - 1) + C * (C + 1)}:
+            return False
+    # schedule kend vs brute visibility, and order
+    S, D, bq, bk = 512, 2, 64, 64
+    perm, _ = oracle.partition(S, D)
+    st, units = oracle.schedule(S, D, 1, 2, 1, True, bq, bk, 2)
+    for u in units:
+        r, i0, k0 = int(u[0]), int(u[3]), int(u[7])
+        rows = perm[r * (S // D) + i0 * bq: r * (S // D) + (i0 + 1) * bq]
+        if k0 != int(rows.max()) // bk + 1:
+            return False
+    work = np.maximum(units[:, 7], units[:, 8])
+    if not (np.diff(work) <= 0).all():
+        return False
+    # forward vs unsharded brute force (GQA, causal)
+    B, S, Hq, Hkv, d, D = 1, 32, 4, 2, 8, 2
+    q = rng.standard_normal((B, S, Hq, d))
+    k = rng.standard_normal((B, S, Hkv, d))
+    v = rng.standard_normal((B, S, Hkv, d))
+    do = rng.standard_normal((B, S, Hq, d))
+    perm, _ = oracle.partition(S, D)
+    qs = inputs.to_shard_major(torch.from_numpy(q), perm, D).numpy()
+    dos = inputs.to_shard_major(torch.from_numpy(do), perm, D).numpy()
+    o, lse = oracle.attn_fwd(qs, k, v, D)
+    o_ref, lse_ref = brute.causal_attention(q, k, v)
+    if np.abs(inputs.from_shard_major(torch.from_numpy(o), perm).numpy() - o_ref).max() > 1e-12:
+        return False
+    if np.abs(inputs.stats_from_shard_major(torch.from_numpy(lse), perm).numpy()
+              - lse_ref).max() > 1e-12:
+        return False
+    # backward vs matrix form
+    g = oracle.attn_bwd(qs, k, v, dos, D)
+    dq_ref, dk_ref, dv_ref = brute.causal_attention_bwd(q, k, v, do)
+    if np.abs(inputs.from_shard_major(torch.from_numpy(g["dq"]), perm).numpy() - dq_ref).max() > 1e-11:
+        return False
+    if np.abs(g["dk"] - dk_ref).max() > 1e-11 or np.abs(g["dv"] - dv_ref).max() > 1e-11:
+        return False
+    return True
+
+
+def test_unmutated_oracle_passes():
+    oracle._load()
+    assert _pins_pass()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name, monkeypatch):
+    lib_path = _build_mutant(tmp_path, name)
+    real = oracle._load()
+    mutant = ctypes.CDLL(lib_path)
+    for fn in ("oracle_partition", "oracle_schedule", "oracle_attn_fwd", "oracle_attn_fwd_rows",
+               "oracle_attn_bwd"):
+        getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
+        getattr(mutant, fn).restype = getattr(real, fn).restype
+    monkeypatch.setattr(oracle, "_lib", mutant)
+    try:
+        ok = _pins_pass()
+    except Exception:
+        ok = False
+    assert not ok, f"mutant {name} slipped through the pins"
