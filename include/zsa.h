@@ -1,0 +1,156 @@
+/*
+ * zsa.h -- C ABI of libzsa: zigzag-sharded causal (GQA) attention on B200 (sm_100a).
+ *
+ * The operation.  A sequence of S positions is cut into 2D equal chunks of
+ * C = S/(2D) positions; logical shard r holds chunk r followed by chunk 2D-1-r
+ * ("Folding Tensor and Sequence Parallelism", summary page, section 2, attention
+ * layer: a zigzag partition balances the causal work across shards).  Every shard's
+ * queries attend to the full, all-gathered K/V (same page and section: an
+ * all-gather rebuilds the full K/V for FlashAttention), with the causal mask taken
+ * on GLOBAL positions ("AutoSP" summary page, section 2.A, step 4: index tensors
+ * such as causal masks are recomputed for the sharded layout).  q head h reads kv
+ * head h / (Hq/Hkv) (grouped-query attention, "Tensor, pipeline e sequence
+ * parallelism", 01 Conceito: 24 q heads over 4 kv heads).  On one GPU all D
+ * shards run in one launch reading one K/V buffer.
+ *
+ *   forward : for shard row (r, j) at position p and q head h,
+ *             s_k = scale * q . k_k for keys k <= p (all k when causal == 0),
+ *             lse = ln sum_k exp(s_k),  O = sum_k exp(s_k - lse) v_k
+ *   backward: the exact gradient of <dO, O>:  Delta = <dO, O>,
+ *             dS_k = P_k (dO . v_k - Delta),  dQ = scale sum_k dS_k k_k,
+ *             dK_k = scale sum dS_k q,  dV_k = sum P_k dO   (sums over every shard
+ *             and every q head of the kv group)
+ *
+ * Layouts (all tensors contiguous, row-major, bf16 unless stated):
+ *   Q, O, dO, dQ : [D][B][2C][Hq][d]   shard-major: shard r's slab is what one rank holds
+ *   K, V, dK, dV : [B][S][Hkv][d]      natural position order (the gathered buffer)
+ *   lse          : fp32 [D][B][Hq][2C] natural logarithm
+ *
+ * Ownership.  The caller owns every buffer: device pointers for tensors and the
+ * workspace, host pointers for zsa_partition's outputs.  The library allocates no
+ * device memory; it caches host-side schedules per shape (thread-safe).
+ *
+ * Asynchrony.  zsa_attn_fwd / zsa_attn_bwd enqueue work on `cuda_stream` (a
+ * cudaStream_t; NULL = legacy default stream) and return without synchronising.
+ * Launch-time CUDA errors return ZSA_ERR_CUDA.  Every device-side wait is bounded;
+ * a wait that gives up records a timeout in the workspace's status word, which
+ * zsa_device_status() reads.
+ *
+ * Errors: every call returns ZSA_OK (0) or a negative ZSA_ERR_* code and never
+ * throws across the ABI.  Argument errors are detected before anything is enqueued.
+ */
+#ifndef ZSA_H
+#define ZSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZSA_API __attribute__((visibility("default")))
+#else
+#define ZSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  ZSA_OK = 0,
+  ZSA_ERR_INVALID = -1,     /* null pointer, non-positive size or scale, misaligned pointer  */
+  ZSA_ERR_SHAPE = -2,       /* S % (2*D*64) != 0, Hq % Hkv != 0                              */
+  ZSA_ERR_UNSUPPORTED = -3, /* head dim not in {64, 128, 256}; device is not sm_100          */
+  ZSA_ERR_WORKSPACE = -4,   /* workspace (or schedule capacity) too small                    */
+  ZSA_ERR_CUDA = -5,        /* a CUDA runtime call failed                                    */
+  ZSA_ERR_TIMEOUT = -6      /* a bounded device-side wait gave up (see zsa_device_status)   */
+};
+
+/* One attention problem.  softmax_scale is applied as an fp32 value (callers usually
+ * pass 1/sqrt(d) rounded to fp32).  causal = 0 gives full (non-causal) attention with
+ * the same layouts. */
+typedef struct {
+  int64_t B, S;
+  int32_t Hq, Hkv, d, D;
+  int32_t causal;
+  float softmax_scale;
+} zsa_problem;
+
+/* Tiling of the forward schedule: block_q query rows per tile, block_k keys per key
+ * tile, `slots` query tiles per work unit (the tiles of one unit share one K/V
+ * stream).  Zero fields mean "library default for d" and are filled in on return. */
+typedef struct {
+  int32_t block_q, block_k, slots;
+} zsa_tiling;
+
+/* One forward work unit: up to two (q tile, q head) slots of shard `shard`, batch
+ * `b`, both q heads in kv group `kv_head`.  k_tile_end = number of key tiles the
+ * slot's rows can see (key tiles 0 .. k_tile_end-1).  An absent second slot has
+ * q_tile1 = q_head1 = -1 and k_tile_end1 = 0. */
+typedef struct {
+  int32_t shard, b, kv_head;
+  int32_t q_tile0, q_head0, q_tile1, q_head1;
+  int32_t k_tile_end0, k_tile_end1;
+} zsa_work;
+
+/*
+ * zsa_partition -- the zigzag index map and the balanced causal tile schedule
+ * (host only, no GPU needed).
+ *   perm_host        [S]  or NULL: perm[r*2C + j] = global position of row j of shard r
+ *   inv_perm_host    [S]  or NULL: inverse of perm
+ *   shard_tiles_host [D]  or NULL: QK^T tile products (block_q x block_k) of shard r,
+ *                         summed over b and q heads; equal for every r (the balance
+ *                         the zigzag provides)
+ *   sched_host       [cap] or NULL: work units in launch order (see zsa_work)
+ *   *n_work_out      number of units (always set when the shape is valid)
+ * Tiling: q tile i of shard r covers rows [i*block_q, (i+1)*block_q) of the shard;
+ * its k_tile_end is (largest position in the tile)/block_k + 1 (causal) or S/block_k.
+ * Units list, per (b, kv head g, shard r), the tile-major slots s = i*G + e (q head
+ * g*G + e) in consecutive runs of `slots`; they are ordered by max k_tile_end
+ * descending, then shard, then run index, then b, then g (all ascending).
+ * Returns ZSA_ERR_WORKSPACE when cap < *n_work_out and sched_host != NULL.
+ */
+ZSA_API int zsa_partition(const zsa_problem* problem, zsa_tiling* tiling, int32_t* perm_host,
+                  int32_t* inv_perm_host, int64_t* shard_tiles_host, zsa_work* sched_host,
+                  int64_t cap, int64_t* n_work_out);
+
+/* Workspace bytes needed by zsa_attn_fwd (pass = 0) or zsa_attn_bwd (pass = 1).
+ * The workspace must be device memory, 256-byte aligned, not shared between calls in
+ * flight.  fwd: status word + the unit table.  bwd: status word + Delta (fp32
+ * [D][B][Hq][2C]) + a dQ accumulator (fp32 [D][B][2C][Hq][d]). */
+ZSA_API int zsa_workspace_bytes(const zsa_problem* problem, int pass, size_t* bytes_out);
+
+/* Forward: o (bf16, Q layout) and lse (fp32 [D][B][Hq][2C]).  q, k, v, o, lse and the
+ * workspace are device pointers, 16-byte aligned. */
+ZSA_API int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
+                 void* o, float* lse, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Backward: dq (Q layout), dk, dv (K layout), all bf16, overwritten (not accumulated).
+ * o and lse must come from zsa_attn_fwd on the same inputs. */
+ZSA_API int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
+                 const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                 void* dv, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Synchronises `cuda_stream`, reads and clears the status word at the start of
+ * `workspace`: ZSA_OK, or ZSA_ERR_TIMEOUT if a device-side wait gave up. */
+ZSA_API int zsa_device_status(void* workspace, void* cuda_stream);
+
+/* Upper bound, in nanoseconds, on any single device-side wait of later launches
+ * (default 2e9).  Test hook: a tiny limit makes the first real wait time out so the
+ * error path can be exercised without hanging anything. */
+ZSA_API int zsa_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Test hook: when `enable` is nonzero, later launches make their MMA-issuing thread
+ * first wait on a barrier that nothing ever arrives at, so the bounded wait must give
+ * up; the launch then tears down (draining its copies and MMAs in flight, releasing
+ * TMEM) and records ZSA_ERR_TIMEOUT in the status word.  Outputs of such a launch are
+ * undefined.  Call with 0 to restore normal operation. */
+ZSA_API int zsa_debug_inject_stall(int enable);
+
+/* Static string for a status code. */
+ZSA_API const char* zsa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZSA_H */

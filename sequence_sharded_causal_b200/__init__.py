@@ -1,0 +1,240 @@
+"""Zigzag-sharded causal (GQA) attention for B200 -- Python binding of libzsa.
+
+The functions named zsa_* mirror the C ABI in include/zsa.h one to one: they only
+marshal arguments (tensor data pointers, the current CUDA stream) and turn status
+codes into exceptions.  Every step of the computation runs in the library's sm_100a
+kernels; there is no CPU or PyTorch fallback: if libzsa.so is missing the calls raise.
+
+attn_fwd / attn_bwd are conveniences that allocate outputs and the workspace through
+PyTorch (device memory only) and then call the same entry points.
+
+Layouts (see include/zsa.h): Q, O, dO, dQ are shard-major [D][B][2C][Hq][d]; K, V, dK,
+dV are natural-order [B][S][Hkv][d]; lse is fp32 [D][B][Hq][2C]; tensors are bf16.
+"""
+import ctypes
+import math
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzsa.so")
+
+ZSA_OK = 0
+ZSA_ERR_INVALID = -1
+ZSA_ERR_SHAPE = -2
+ZSA_ERR_UNSUPPORTED = -3
+ZSA_ERR_WORKSPACE = -4
+ZSA_ERR_CUDA = -5
+ZSA_ERR_TIMEOUT = -6
+
+EXPORTED = ("zsa_partition", "zsa_workspace_bytes", "zsa_attn_fwd", "zsa_attn_bwd",
+            "zsa_device_status", "zsa_set_wait_limit_ns", "zsa_debug_inject_stall",
+            "zsa_status_string")
+
+
+class zsa_problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("S", ctypes.c_int64), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("causal", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+
+
+class zsa_tiling(ctypes.Structure):
+    _fields_ = [("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32), ("slots", ctypes.c_int32)]
+
+
+class zsa_work(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("shard", "b", "kv_head", "q_tile0", "q_head0",
+                                              "q_tile1", "q_head1", "k_tile_end0", "k_tile_end1")]
+
+
+class ZsaError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libzsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sequence_sharded_causal_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER
+        vp = ctypes.c_void_p
+        L.zsa_partition.argtypes = [P(zsa_problem), P(zsa_tiling), vp, vp, vp, vp, ctypes.c_int64,
+                                    P(ctypes.c_int64)]
+        L.zsa_workspace_bytes.argtypes = [P(zsa_problem), ctypes.c_int, P(ctypes.c_size_t)]
+        L.zsa_attn_fwd.argtypes = [P(zsa_problem), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.zsa_attn_bwd.argtypes = [P(zsa_problem)] + [vp] * 10 + [ctypes.c_size_t, vp]
+        L.zsa_device_status.argtypes = [vp, vp]
+        L.zsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.zsa_debug_inject_stall.argtypes = [ctypes.c_int]
+        L.zsa_status_string.argtypes = [ctypes.c_int]
+        L.zsa_status_string.restype = ctypes.c_char_p
+        for name in EXPORTED[:-1]:
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().zsa_status_string(int(status)).decode()
+
+
+def _check(rc, where):
+    if rc != ZSA_OK:
+        raise ZsaError(rc, where)
+
+
+def make_problem(B, S, Hq, Hkv, d, D, causal=True, scale=None):
+    if scale is None:
+        scale = float(np.float32(1.0 / math.sqrt(d)))
+    return zsa_problem(int(B), int(S), int(Hq), int(Hkv), int(d), int(D), int(bool(causal)),
+                       float(scale))
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ C ABI mirrors
+
+def zsa_partition(problem, block_q=0, block_k=0, slots=0, want_schedule=True):
+    """Zigzag map + forward schedule (host only).
+
+    Returns dict: perm, inv_perm (int32 [S]), shard_tiles (int64 [D]), sched (int32
+    [n][9]: shard, b, kv_head, q_tile0, q_head0, q_tile1, q_head1, k_tile_end0,
+    k_tile_end1) and the tiling actually used.
+    """
+    t = zsa_tiling(block_q, block_k, slots)
+    S, D = int(problem.S), int(problem.D)
+    perm = np.empty(S, np.int32)
+    inv = np.empty(S, np.int32)
+    st = np.empty(D, np.int64)
+    n = ctypes.c_int64(0)
+    _check(lib().zsa_partition(ctypes.byref(problem), ctypes.byref(t), perm.ctypes.data,
+                               inv.ctypes.data, st.ctypes.data, None, 0, ctypes.byref(n)),
+           "zsa_partition")
+    sched = None
+    if want_schedule:
+        sched = np.empty((n.value, 9), np.int32)
+        _check(lib().zsa_partition(ctypes.byref(problem), ctypes.byref(t), None, None, None,
+                                   sched.ctypes.data, n.value, ctypes.byref(n)), "zsa_partition")
+    return dict(perm=perm, inv_perm=inv, shard_tiles=st, sched=sched,
+                tiling=(t.block_q, t.block_k, t.slots))
+
+
+def zsa_workspace_bytes(problem, pass_):
+    out = ctypes.c_size_t(0)
+    _check(lib().zsa_workspace_bytes(ctypes.byref(problem), int(pass_), ctypes.byref(out)),
+           "zsa_workspace_bytes")
+    return out.value
+
+
+def zsa_attn_fwd(problem, q, k, v, o, lse, workspace, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().zsa_attn_fwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                              _ptr(lse), _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "zsa_attn_fwd")
+
+
+def zsa_attn_bwd(problem, q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes=None,
+                 stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().zsa_attn_bwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                              _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                              _ptr(workspace), int(ws_bytes), _stream(stream)), "zsa_attn_bwd")
+
+
+def zsa_device_status(workspace, stream=None):
+    """Synchronise and return the device status word (0 or ZSA_ERR_TIMEOUT); clears it."""
+    return lib().zsa_device_status(_ptr(workspace), _stream(stream))
+
+
+def zsa_set_wait_limit_ns(limit_ns):
+    _check(lib().zsa_set_wait_limit_ns(int(limit_ns)), "zsa_set_wait_limit_ns")
+
+
+def zsa_debug_inject_stall(enable):
+    _check(lib().zsa_debug_inject_stall(int(bool(enable))), "zsa_debug_inject_stall")
+
+
+def zsa_status_string(status):
+    return status_string(status)
+
+
+# ------------------------------------------------------------------ conveniences
+
+def _check_tensor(x, shape, dtype, name):
+    import torch
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(x.shape) != tuple(shape) or x.dtype != dtype or not x.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got "
+                         f"{x.dtype} {tuple(x.shape)} contiguous={x.is_contiguous()}")
+
+
+def _shapes(problem):
+    B, S, Hq, Hkv, d, D = (int(problem.B), int(problem.S), int(problem.Hq), int(problem.Hkv),
+                           int(problem.d), int(problem.D))
+    return (D, B, S // D, Hq, d), (B, S, Hkv, d), (D, B, Hq, S // D)
+
+
+def attn_fwd(q, k, v, D, causal=True, scale=None, workspace=None):
+    """O, lse = attention(Q, K, V) with all D zigzag shards in one launch."""
+    import torch
+    Dq, B, twoC, Hq, d = q.shape
+    S = Dq * twoC
+    problem = make_problem(B, S, Hq, k.shape[2], d, D, causal, scale)
+    qs, ks, ls = _shapes(problem)
+    _check_tensor(q, qs, torch.bfloat16, "q")
+    _check_tensor(k, ks, torch.bfloat16, "k")
+    _check_tensor(v, ks, torch.bfloat16, "v")
+    o = torch.empty_like(q)
+    lse = torch.empty(ls, dtype=torch.float32, device=q.device)
+    nbytes = zsa_workspace_bytes(problem, 0)
+    if workspace is None or workspace.numel() * workspace.element_size() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    zsa_attn_fwd(problem, q, k, v, o, lse, workspace)
+    return o, lse
+
+
+def attn_bwd(q, k, v, o, lse, do, D, causal=True, scale=None, workspace=None):
+    """dQ, dK, dV of <dO, O> (dK/dV summed over all shards and the q heads of a group)."""
+    import torch
+    Dq, B, twoC, Hq, d = q.shape
+    S = Dq * twoC
+    problem = make_problem(B, S, Hq, k.shape[2], d, D, causal, scale)
+    qs, ks, ls = _shapes(problem)
+    for name, x, shp in (("q", q, qs), ("k", k, ks), ("v", v, ks), ("o", o, qs), ("do", do, qs)):
+        _check_tensor(x, shp, torch.bfloat16, name)
+    _check_tensor(lse, ls, torch.float32, "lse")
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    nbytes = zsa_workspace_bytes(problem, 1)
+    if workspace is None or workspace.numel() * workspace.element_size() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    zsa_attn_bwd(problem, q, k, v, o, lse, do, dq, dk, dv, workspace)
+    return dq, dk, dv

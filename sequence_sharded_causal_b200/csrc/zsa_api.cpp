@@ -1,0 +1,299 @@
+// zsa_api.cpp -- the C ABI declared in include/zsa.h.
+//
+// Argument validation happens here, before anything is enqueued; every entry point
+// returns a status code and nothing throws across the ABI.  The library allocates no
+// device memory: the forward's unit table travels in the caller's workspace, copied
+// from a pinned host copy that is cached per shape.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <tuple>
+
+#include "../../include/zsa.h"
+#include "zsa_kernels.h"
+#include "zsa_schedule.h"
+
+namespace {
+
+using zsa::Schedule;
+
+constexpr size_t kStatusBytes = 256;
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_inject_stall{0};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_problem(const zsa_problem* p) {
+  if (!p) return ZSA_ERR_INVALID;
+  if (p->B <= 0 || p->S <= 0 || p->Hq <= 0 || p->Hkv <= 0 || p->d <= 0 || p->D <= 0)
+    return ZSA_ERR_INVALID;
+  if (!(p->softmax_scale > 0.0f) || !std::isfinite(p->softmax_scale)) return ZSA_ERR_INVALID;
+  if (p->causal != 0 && p->causal != 1) return ZSA_ERR_INVALID;
+  if (p->Hq % p->Hkv != 0) return ZSA_ERR_SHAPE;
+  if (p->S % (2 * int64_t(p->D) * 64) != 0) return ZSA_ERR_SHAPE;
+  if (p->B * p->S >= (int64_t(1) << 31)) return ZSA_ERR_SHAPE;  // TMA row coordinates are int32
+  return ZSA_OK;
+}
+
+int check_device_problem(const zsa_problem* p) {
+  int rc = check_problem(p);
+  if (rc) return rc;
+  if (p->d != 64 && p->d != 128 && p->d != 256) return ZSA_ERR_UNSUPPORTED;
+  int32_t bq, bk, slots;
+  zsa::fwd_tiling(p->d, &bq, &bk, &slots);
+  if (p->S / bk >= 65536) return ZSA_ERR_SHAPE;  // key-tile counts are packed in 16 bits
+  return ZSA_OK;
+}
+
+bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
+
+int check_sm100() {
+  static std::mutex mu;
+  static std::map<int, int> verdict;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ZSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = verdict.find(dev);
+  if (it != verdict.end()) return it->second;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return ZSA_ERR_CUDA;
+  int v = (major == 10 && minor == 0) ? ZSA_OK : ZSA_ERR_UNSUPPORTED;
+  verdict[dev] = v;
+  return v;
+}
+
+// ------------------------------------------------------------------ schedule cache
+struct CachedSchedule {
+  Schedule sched;
+  zsa::DevUnit* pinned = nullptr;  // page-locked copy of sched.units (or nullptr)
+  ~CachedSchedule() {
+    if (pinned) cudaFreeHost(pinned);
+  }
+};
+
+using SchedKey = std::tuple<int64_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t>;
+
+std::shared_ptr<CachedSchedule> get_schedule(int64_t S, int32_t D, int32_t B, int32_t Hq,
+                                             int32_t Hkv, int32_t causal, int32_t bq, int32_t bk,
+                                             int32_t slots, bool want_pinned) {
+  static std::mutex mu;
+  static std::map<SchedKey, std::shared_ptr<CachedSchedule>> cache;
+  SchedKey key{S, D, B, Hq, Hkv, causal, bq, bk, slots};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end() && (!want_pinned || it->second->pinned)) return it->second;
+  }
+  auto e = std::make_shared<CachedSchedule>();
+  if (!zsa::build_schedule(S, D, B, Hq, Hkv, causal, bq, bk, slots, &e->sched)) return nullptr;
+  if (want_pinned) {
+    const size_t bytes = e->sched.units.size() * sizeof(zsa::DevUnit);
+    void* h = nullptr;
+    if (cudaHostAlloc(&h, bytes ? bytes : 1, cudaHostAllocDefault) != cudaSuccess) return nullptr;
+    std::memcpy(h, e->sched.units.data(), bytes);
+    e->pinned = static_cast<zsa::DevUnit*>(h);
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  auto& slot = cache[key];
+  if (!slot || (want_pinned && !slot->pinned)) slot = e;
+  return slot;
+}
+
+size_t fwd_workspace(const zsa_problem* p) {
+  int32_t bq, bk, slots;
+  zsa::fwd_tiling(p->d, &bq, &bk, &slots);
+  const int64_t T = (p->S / p->D) / bq;
+  const int64_t G = p->Hq / p->Hkv;
+  const int64_t runs = (T * G + slots - 1) / slots;
+  const int64_t units = p->B * p->Hkv * p->D * runs;
+  return kStatusBytes + align256(size_t(units) * sizeof(zsa::DevUnit));
+}
+
+size_t bwd_workspace(const zsa_problem* p) {
+  const size_t stats = size_t(p->B) * p->S * p->Hq * sizeof(float);       // Delta
+  const size_t dqacc = size_t(p->B) * p->S * p->Hq * p->d * sizeof(float);
+  return kStatusBytes + align256(stats) + align256(dqacc);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* zsa_status_string(int status) {
+  switch (status) {
+    case ZSA_OK: return "ok";
+    case ZSA_ERR_INVALID: return "invalid argument";
+    case ZSA_ERR_SHAPE: return "unsupported shape (S % (2*D*64), Hq % Hkv or size limits)";
+    case ZSA_ERR_UNSUPPORTED: return "unsupported head dim or device (needs sm_100)";
+    case ZSA_ERR_WORKSPACE: return "workspace or schedule capacity too small";
+    case ZSA_ERR_CUDA: return "CUDA runtime error";
+    case ZSA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int zsa_debug_inject_stall(int enable) {
+  g_inject_stall.store(enable ? 1 : 0);
+  return ZSA_OK;
+}
+
+int zsa_set_wait_limit_ns(uint64_t limit_ns) {
+  g_wait_limit_ns.store(limit_ns);
+  return ZSA_OK;
+}
+
+int zsa_partition(const zsa_problem* problem, zsa_tiling* tiling, int32_t* perm_host,
+                  int32_t* inv_perm_host, int64_t* shard_tiles_host, zsa_work* sched_host,
+                  int64_t cap, int64_t* n_work_out) {
+  int rc = check_problem(problem);
+  if (rc) return rc;
+  if (!tiling) return ZSA_ERR_INVALID;
+  int32_t bq = tiling->block_q, bk = tiling->block_k, slots = tiling->slots;
+  if (bq == 0 || bk == 0 || slots == 0) {
+    int32_t dq, dk, ds;
+    zsa::fwd_tiling(problem->d, &dq, &dk, &ds);
+    if (bq == 0) bq = dq;
+    if (bk == 0) bk = dk;
+    if (slots == 0) slots = ds;
+  }
+  const int64_t S = problem->S;
+  const int32_t D = problem->D;
+  if (bq < 0 || bk < 0 || (slots != 1 && slots != 2)) return ZSA_ERR_INVALID;
+  if ((S / D) % bq != 0 || S % bk != 0) return ZSA_ERR_SHAPE;
+  if (S / bk >= 65536) return ZSA_ERR_SHAPE;
+  tiling->block_q = bq;
+  tiling->block_k = bk;
+  tiling->slots = slots;
+  const int64_t C = S / (2 * int64_t(D));
+  if (perm_host || inv_perm_host) {
+    for (int32_t r = 0; r < D; ++r)
+      for (int64_t j = 0; j < 2 * C; ++j) {
+        const int64_t pos = zsa::zigzag_pos(C, D, r, j);
+        if (perm_host) perm_host[r * 2 * C + j] = int32_t(pos);
+        if (inv_perm_host) inv_perm_host[pos] = int32_t(r * 2 * C + j);
+      }
+  }
+  if (!shard_tiles_host && !sched_host && !n_work_out) return ZSA_OK;
+  auto cs = get_schedule(S, D, int32_t(problem->B), problem->Hq, problem->Hkv, problem->causal, bq,
+                         bk, slots, false);
+  if (!cs) return ZSA_ERR_SHAPE;
+  const Schedule& sc = cs->sched;
+  if (shard_tiles_host)
+    for (int32_t r = 0; r < D; ++r) shard_tiles_host[r] = sc.shard_tiles[size_t(r)];
+  const int64_t n = int64_t(sc.units.size());
+  if (n_work_out) *n_work_out = n;
+  if (sched_host) {
+    if (cap < n) return ZSA_ERR_WORKSPACE;
+    for (int64_t i = 0; i < n; ++i) {
+      const zsa::DevUnit& u = sc.units[size_t(i)];
+      zsa_work& w = sched_host[i];
+      w.shard = u.r; w.b = u.b; w.kv_head = u.g;
+      w.q_tile0 = u.tile0; w.q_head0 = u.head0; w.q_tile1 = u.tile1; w.q_head1 = u.head1;
+      w.k_tile_end0 = u.kend & 0xFFFF;
+      w.k_tile_end1 = (u.kend >> 16) & 0xFFFF;
+    }
+  }
+  return ZSA_OK;
+}
+
+int zsa_workspace_bytes(const zsa_problem* problem, int pass, size_t* bytes_out) {
+  int rc = check_device_problem(problem);
+  if (rc) return rc;
+  if (!bytes_out || (pass != 0 && pass != 1)) return ZSA_ERR_INVALID;
+  *bytes_out = pass == 0 ? fwd_workspace(problem) : bwd_workspace(problem);
+  return ZSA_OK;
+}
+
+int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
+                 void* o, float* lse, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  int rc = check_device_problem(problem);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse || !workspace) return ZSA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return ZSA_ERR_INVALID;
+  if (ws_bytes < fwd_workspace(problem)) return ZSA_ERR_WORKSPACE;
+  rc = check_sm100();
+  if (rc) return rc;
+  int32_t bq, bk, slots;
+  zsa::fwd_tiling(problem->d, &bq, &bk, &slots);
+  auto cs = get_schedule(problem->S, problem->D, int32_t(problem->B), problem->Hq, problem->Hkv,
+                         problem->causal, bq, bk, slots, true);
+  if (!cs) return ZSA_ERR_CUDA;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t table = cs->sched.units.size() * sizeof(zsa::DevUnit);
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  if (table &&
+      cudaMemcpyAsync(ws + kStatusBytes, cs->pinned, table, cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess)
+    return ZSA_ERR_CUDA;
+  zsa::FwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.units = reinterpret_cast<const zsa::DevUnit*>(ws + kStatusBytes);
+  a.n_units = int32_t(cs->sched.units.size());
+  a.S = problem->S; a.B = int32_t(problem->B); a.Hq = problem->Hq; a.Hkv = problem->Hkv;
+  a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
+  a.scale = problem->softmax_scale;
+  a.status = reinterpret_cast<int*>(ws);
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.inject_stall = g_inject_stall.load();
+  if (zsa::launch_fwd(a, stream) != int(cudaSuccess)) return ZSA_ERR_CUDA;
+  return ZSA_OK;
+}
+
+int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
+                 const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                 void* workspace, size_t ws_bytes, void* cuda_stream) {
+  int rc = check_device_problem(problem);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return ZSA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return ZSA_ERR_INVALID;
+  if (ws_bytes < bwd_workspace(problem)) return ZSA_ERR_WORKSPACE;
+  rc = check_sm100();
+  if (rc) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t stats = size_t(problem->B) * problem->S * problem->Hq * sizeof(float);
+  zsa::BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.delta = reinterpret_cast<float*>(ws + kStatusBytes);
+  a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes + align256(stats));
+  a.S = problem->S; a.B = int32_t(problem->B); a.Hq = problem->Hq; a.Hkv = problem->Hkv;
+  a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
+  a.scale = problem->softmax_scale;
+  a.status = reinterpret_cast<int*>(ws);
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  a.inject_stall = g_inject_stall.load();
+  const int e = zsa::launch_bwd(a, stream);
+  if (e == int(cudaErrorNotSupported)) return ZSA_ERR_UNSUPPORTED;
+  if (e != int(cudaSuccess)) return ZSA_ERR_CUDA;
+  return ZSA_OK;
+}
+
+int zsa_device_status(void* workspace, void* cuda_stream) {
+  if (!workspace) return ZSA_ERR_INVALID;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  int st = 0;
+  if (cudaMemcpyAsync(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return ZSA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  if (st == 0) return ZSA_OK;
+  if (cudaMemsetAsync(workspace, 0, sizeof(int), stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  return ZSA_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,503 @@
+// zsa_fwd.cu -- forward kernel (K1): zigzag-sharded causal GQA attention on sm_100a.
+//
+// Method: every shard's queries attend FlashAttention-style to the full gathered K/V
+// ("Folding Tensor and Sequence Parallelism" summary, section 2, attention layer), the
+// causal mask on global positions ("AutoSP" summary, section 2.A step 4), q heads
+// sharing kv heads ("Tensor, pipeline e sequence parallelism", 01 Conceito).  The
+// pages give no kernel design; this one is built for the B200:
+//
+//  * persistent CTAs, one per SM, walk the host-built unit table (units sorted by
+//    work, longest first, assigned in snake order);
+//  * a unit is up to NSLOT (q tile, q head) slots of 128 query rows that share one K/V
+//    stream: two q heads of one kv group (GQA) or two adjacent q tiles (MHA), so a
+//    K/V tile fetched once feeds 2 x 128 rows of MMAs;
+//  * warp roles: 4 softmax warps per slot (one TMEM lane = one query row per thread),
+//    1 TMA producer warp, 1 MMA warp (one thread issues tcgen05.mma);
+//  * S = Q K^T goes to TMEM (128 x BK fp32); the softmax warps read it, apply the
+//    global-position mask, keep a running max (rescaling O in TMEM only when the max
+//    grows by more than 2^8) and write P as bf16 back over S; O += P V is a TMEM-A
+//    MMA (P from TMEM, V from shared memory as an MN-major operand);
+//  * shared memory: Q tiles resident for the unit, a K ring and a V ring of ST stages,
+//    all 128B-swizzled TMA tiles; TMEM: S0 | S1 | O0 | O1 (512 columns at d = 128).
+// MMA issue order per key tile n: PV0(n), QK0(n+1), PV1(n), QK1(n+1), so each slot's
+// softmax overlaps the other slot's two MMAs.  QK_s(n+1) overwrites the columns P_s(n)
+// lives in, so it is issued only after PV_s(n) has completed (pv_done barrier).
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "zsa_kernels.h"
+#include "zsa_ptx.cuh"
+#include "zsa_tma_host.h"
+
+namespace zsa {
+namespace {
+
+template <int HD>
+struct FwdCfg {
+  static constexpr int NSLOT = HD <= 128 ? 2 : 1;
+  static constexpr int BQ = 128;
+  static constexpr int BK = HD <= 128 ? 128 : 64;
+  static constexpr int ST = HD == 64 ? 4 : 2;
+  static constexpr int KB = HD / 64;                  // 64-wide (128-byte) d blocks
+  static constexpr int Q_BYTES = BQ * HD * 2;
+  static constexpr int KV_BYTES = BK * HD * 2;
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_K = SMEM_Q + NSLOT * Q_BYTES;
+  static constexpr int SMEM_V = SMEM_K + ST * KV_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_V + ST * KV_BYTES;
+  static constexpr int NWARP_SOFTMAX = 4 * NSLOT;
+  static constexpr int WARP_LOAD = NWARP_SOFTMAX;
+  static constexpr int WARP_MMA = NWARP_SOFTMAX + 1;
+  static constexpr int NTHREADS = (NWARP_SOFTMAX + 2) * 32;
+  static constexpr uint32_t TM_COLS = 512;
+  __device__ static constexpr uint32_t tm_s(int s) { return uint32_t(s * 128); }
+  __device__ static constexpr uint32_t tm_o(int s) { return uint32_t(256 + s * HD); }
+  static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
+  static_assert(256 + NSLOT * HD <= 512, "TMEM budget");
+};
+
+struct FwdParams {
+  const DevUnit* units;
+  int32_t n_units;
+  __nv_bfloat16* o;
+  float* lse;
+  int64_t S, C;
+  int32_t B, Hq, Hkv, D, causal;
+  float scale_log2;
+  int* status;
+  uint64_t wait_limit_ns;
+  int inject_stall;
+};
+
+struct FwdBars {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t drain;
+  uint64_t never;  // test hook: no one ever arrives here
+};
+
+struct UnitInfo {
+  int32_t r, b, g;
+  int32_t tile[2], head[2], kend[2];
+  int32_t nmax;
+};
+
+__device__ __forceinline__ UnitInfo load_unit(const DevUnit* units, int idx) {
+  const int4* p = reinterpret_cast<const int4*>(units + idx);
+  int4 a = __ldg(p), c = __ldg(p + 1);
+  UnitInfo u;
+  u.r = a.x; u.b = a.y; u.g = a.z;
+  u.tile[0] = a.w; u.head[0] = c.x; u.tile[1] = c.y; u.head[1] = c.z;
+  u.kend[0] = c.w & 0xFFFF;
+  u.kend[1] = (c.w >> 16) & 0xFFFF;
+  u.nmax = u.kend[0] > u.kend[1] ? u.kend[0] : u.kend[1];
+  return u;
+}
+
+// k-th unit of this CTA in snake order over stripes of gridDim.x units; -1 when done.
+__device__ __forceinline__ int unit_index(int k, int n_units) {
+  const int grid = int(gridDim.x);
+  const int idx = k * grid + ((k & 1) ? (grid - 1 - int(blockIdx.x)) : int(blockIdx.x));
+  return idx < n_units ? idx : -1;
+}
+
+// Every lane polls; the outcome is made warp-uniform so .sync.aligned TMEM ops that
+// follow are executed by the full warp or by none of it.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  bool ok = mbar_wait(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
+    zsa_fwd_kernel(const __grid_constant__ CUtensorMap map_q,
+                   const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v, const FwdParams prm) {
+  using Cfg = FwdCfg<HD>;
+  constexpr int NSLOT = Cfg::NSLOT, BK = Cfg::BK, ST = Cfg::ST, KB = Cfg::KB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ FwdBars bars;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  const int warp = int(warp_id()), lane = int(lane_id());
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_empty[s], 1);
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.p_full[s], 4);
+      mbar_init(&bars.pv_done[s], 1);
+      mbar_init(&bars.o_full[s], 1);
+      mbar_init(&bars.o_empty[s], 4);
+    }
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&bars.k_full[s], 1);
+      mbar_init(&bars.k_empty[s], 1);
+      mbar_init(&bars.v_full[s], 1);
+      mbar_init(&bars.v_empty[s], 1);
+    }
+    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.never, 1);
+    fence_mbar_init();
+  }
+  if (warp == Cfg::WARP_MMA) {
+    tmem_alloc(&tmem_base_s, Cfg::TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == Cfg::WARP_LOAD && lane == 0) {
+    tma_prefetch_desc(&map_q);
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  const WaitCtx wctx{&abort_s, prm.status, prm.wait_limit_ns};
+  const uint32_t sQ = smem_u32(smem + Cfg::SMEM_Q);
+  const uint32_t sK = smem_u32(smem + Cfg::SMEM_K);
+  const uint32_t sV = smem_u32(smem + Cfg::SMEM_V);
+  const int64_t twoC = 2 * prm.C;
+
+  if (warp == Cfg::WARP_LOAD) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv_it = 0;
+      uint32_t q_fills[2] = {0, 0};
+      uint32_t k_fills[ST], v_fills[ST];
+      for (int st = 0; st < ST; ++st) k_fills[st] = v_fills[st] = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = unit_index(k, prm.n_units);
+        if (idx < 0) break;
+        const UnitInfo u = load_unit(prm.units, idx);
+        for (int s = 0; s < NSLOT && ok; ++s) {
+          if (u.kend[s] == 0) continue;
+          if (q_fills[s] > 0) ok = mbar_wait(&bars.q_empty[s], (q_fills[s] - 1) & 1, wctx);
+          if (!ok) break;
+          mbar_expect_tx(&bars.q_full[s], Cfg::Q_BYTES);
+          const int32_t row0 = int32_t((int64_t(u.r) * prm.B + u.b) * twoC + int64_t(u.tile[s]) * 128);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(smem + Cfg::SMEM_Q + s * Cfg::Q_BYTES + kb * 128 * 128, &map_q,
+                        &bars.q_full[s], kb * 64, u.head[s], row0);
+          ++q_fills[s];
+        }
+        for (int n = 0; n < u.nmax && ok; ++n) {
+          const uint32_t it = kv_it + uint32_t(n);
+          const int st = int(it % ST);
+          const uint32_t use = it / ST;
+          const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(n) * BK);
+          if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, wctx);
+          if (!ok) break;
+          mbar_expect_tx(&bars.k_full[st], Cfg::KV_BYTES);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128, &map_k,
+                        &bars.k_full[st], kb * 64, u.g, key0);
+          ++k_fills[st];
+          if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, wctx);
+          if (!ok) break;
+          mbar_expect_tx(&bars.v_full[st], Cfg::KV_BYTES);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128, &map_v,
+                        &bars.v_full[st], kb * 64, u.g, key0);
+          ++v_fills[st];
+        }
+        kv_it += uint32_t(u.nmax);
+      }
+      if (!ok) {
+        // Teardown after an abort: wait (bounded) for every fill still in flight.
+        const uint64_t lim = 1000000000ull;
+        for (int s = 0; s < NSLOT; ++s)
+          if (q_fills[s] > 0) mbar_drain(&bars.q_full[s], (q_fills[s] - 1) & 1, lim);
+        for (int st = 0; st < ST; ++st) {
+          if (k_fills[st] > 0) mbar_drain(&bars.k_full[st], (k_fills[st] - 1) & 1, lim);
+          if (v_fills[st] > 0) mbar_drain(&bars.v_full[st], (v_fills[st] - 1) & 1, lim);
+        }
+      }
+    }
+  } else if (warp == Cfg::WARP_MMA) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16(128, BK, false, false);
+      const uint32_t idesc_pv = idesc_bf16(128, HD, false, true);
+      uint32_t kv_it = 0;
+      uint32_t q_ph[2] = {0, 0}, p_ph[2] = {0, 0}, pv_ph[2] = {0, 0}, oe_ph[2] = {0, 0};
+      bool pv_pending[2] = {false, false}, o_pending[2] = {false, false};
+      bool ok = true;
+      if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
+      auto issue_qk = [&](int s, int st) {
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t a = sdesc_sw128(sQ + s * Cfg::Q_BYTES + kb * 128 * 128 + ks * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(sK + st * Cfg::KV_BYTES + kb * BK * 128 + ks * 32, 16, 1024);
+            mma_ss(tmem + Cfg::tm_s(s), a, b, idesc_qk, (kb | ks) != 0);
+          }
+      };
+      auto issue_pv = [&](int s, int st, int n) {
+#pragma unroll
+        for (int ks = 0; ks < BK / 16; ++ks) {
+          const uint64_t b = sdesc_sw128(sV + st * Cfg::KV_BYTES + ks * 2048, BK * 128, 1024);
+          mma_ts(tmem + Cfg::tm_o(s), tmem + Cfg::tm_s(s) + ks * 8, b, idesc_pv, (n > 0) || (ks > 0));
+        }
+      };
+      for (int k = 0; ok; ++k) {
+        const int idx = unit_index(k, prm.n_units);
+        if (idx < 0) break;
+        const UnitInfo u = load_unit(prm.units, idx);
+        for (int s = 0; s < NSLOT && ok; ++s) {
+          if (u.kend[s] == 0) continue;
+          ok = mbar_wait(&bars.q_full[s], q_ph[s], wctx);
+          q_ph[s] ^= 1;
+        }
+        if (!ok) break;
+        // prologue: S_s(0) = Q_s K(0)^T
+        {
+          const int st = int(kv_it % ST);
+          ok = mbar_wait(&bars.k_full[st], (kv_it / ST) & 1, wctx);
+          if (!ok) break;
+          for (int s = 0; s < NSLOT && ok; ++s) {
+            if (u.kend[s] == 0) continue;
+            if (pv_pending[s]) {
+              ok = mbar_wait(&bars.pv_done[s], pv_ph[s], wctx);
+              pv_ph[s] ^= 1;
+              pv_pending[s] = false;
+              if (!ok) break;
+            }
+            tc_fence_after();
+            issue_qk(s, st);
+            mma_commit(&bars.s_full[s]);
+            if (u.kend[s] == 1) mma_commit(&bars.q_empty[s]);
+          }
+          if (!ok) break;
+          mma_commit(&bars.k_empty[st]);
+        }
+        for (int n = 0; n < u.nmax && ok; ++n) {
+          const uint32_t it = kv_it + uint32_t(n);
+          const int st = int(it % ST);
+          const int st1 = int((it + 1) % ST);
+          ok = mbar_wait(&bars.v_full[st], (it / ST) & 1, wctx);
+          bool knext = false;
+          for (int s = 0; s < NSLOT && ok; ++s) {
+            if (n >= u.kend[s]) continue;
+            ok = mbar_wait(&bars.p_full[s], p_ph[s], wctx);
+            p_ph[s] ^= 1;
+            if (ok && n == 0 && o_pending[s]) {
+              ok = mbar_wait(&bars.o_empty[s], oe_ph[s], wctx);
+              oe_ph[s] ^= 1;
+              o_pending[s] = false;
+            }
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(s, st, n);
+            mma_commit(&bars.pv_done[s]);
+            pv_pending[s] = true;
+            if (n == u.kend[s] - 1) {
+              mma_commit(&bars.o_full[s]);
+              o_pending[s] = true;
+            }
+            if (n + 1 < u.kend[s]) {
+              if (!knext) {
+                ok = mbar_wait(&bars.k_full[st1], ((it + 1) / ST) & 1, wctx);
+                knext = true;
+              }
+              if (ok) ok = mbar_wait(&bars.pv_done[s], pv_ph[s], wctx);
+              pv_ph[s] ^= 1;
+              pv_pending[s] = false;
+              if (!ok) break;
+              tc_fence_after();
+              issue_qk(s, st1);
+              mma_commit(&bars.s_full[s]);
+              if (n + 1 == u.kend[s] - 1) mma_commit(&bars.q_empty[s]);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bars.v_empty[st]);
+          if (knext) mma_commit(&bars.k_empty[st1]);
+        }
+        kv_it += uint32_t(u.nmax);
+      }
+      // Teardown: every MMA issued so far completes before TMEM is released.
+      mma_commit(&bars.drain);
+      mbar_drain(&bars.drain, 0, 1000000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int s = warp / 4;            // slot
+    const int qw = warp % 4;           // TMEM lane quarter
+    const int row = qw * 32 + lane;    // query row within the tile = TMEM lane
+    const uint32_t lane_addr = uint32_t(qw * 32) << 16;
+    const uint32_t tS = tmem + Cfg::tm_s(s) + lane_addr;
+    const uint32_t tO = tmem + Cfg::tm_o(s) + lane_addr;
+    uint32_t s_ph = 0, o_ph = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = unit_index(k, prm.n_units);
+      if (idx < 0) break;
+      const UnitInfo u = load_unit(prm.units, idx);
+      if (u.kend[s] == 0) continue;
+      const int64_t j = int64_t(u.tile[s]) * 128 + row;             // row within the shard
+      const int64_t pos = j < prm.C ? int64_t(u.r) * prm.C + j
+                                    : int64_t(2 * prm.D - 1 - u.r) * prm.C + (j - prm.C);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int n = 0; n < u.kend[s]; ++n) {
+        ok = warp_wait(&bars.s_full[s], s_ph, wctx);
+        s_ph ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[BK / 32][32];
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
+        tmem_ld_wait();
+        const int64_t key0 = int64_t(n) * BK;
+        const bool masked = prm.causal && (key0 + BK - 1 > pos);
+        float mt = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float x = __uint_as_float(sr[c][e]) * prm.scale_log2;
+            if (masked && key0 + c * 32 + e > pos) x = -INFINITY;
+            sr[c][e] = __float_as_uint(x);
+            mt = fmaxf(mt, x);
+          }
+        const float m_new = fmaxf(m_run, mt);
+        if (m_new > m_run + 8.0f) {
+          if (n > 0) {
+            // O was accumulated against the old max: scale it (and l) down.
+            const float alpha = ex2_approx(m_run - m_new);
+            l_run *= alpha;
+#pragma unroll 1
+            for (int c = 0; c < HD / 32; ++c) {
+              uint32_t orow[32];
+              tmem_ld32(tO + c * 32, orow);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+              tmem_st32(tO + c * 32, orow);
+            }
+          }
+          m_run = m_new;
+        }
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(__uint_as_float(sr[c][2 * e]) - m_run);
+            const float p1 = ex2_approx(__uint_as_float(sr[c][2 * e + 1]) - m_run);
+            lsum += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);     // P (bf16 pairs) over the S columns already read
+        }
+        l_run += lsum;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[s]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, lse
+      ok = warp_wait(&bars.o_full[s], o_ph, wctx);
+      o_ph ^= 1;
+      if (!ok) break;
+      tc_fence_after();
+      const float inv_l = 1.0f / l_run;
+      const int64_t grow = (int64_t(u.r) * prm.B + u.b) * twoC + j;    // shard-major row
+      __nv_bfloat16* orow_g = prm.o + (grow * prm.Hq + u.head[s]) * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t orow[32];
+        tmem_ld32(tO + c * 32, orow);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(orow[2 * e]) * inv_l,
+                              __uint_as_float(orow[2 * e + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      }
+      prm.lse[((int64_t(u.r) * prm.B + u.b) * prm.Hq + u.head[s]) * twoC + j] =
+          (m_run + log2f(l_run)) * 0.69314718055994530942f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.o_empty[s]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == Cfg::WARP_MMA) tmem_dealloc(tmem, Cfg::TM_COLS);
+}
+
+template <int HD>
+int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
+  using Cfg = FwdCfg<HD>;
+  const int64_t rows = a.S * a.B;  // D * B * 2C shard-major rows
+  CUtensorMap mq, mk, mv;
+  {
+    const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hq), uint64_t(rows)};
+    const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hq) * HD * 2};
+    const uint32_t box[3] = {64, 1, 128};
+    if (!make_map_bf16_sw128(&mq, a.q, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+  }
+  {
+    const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), uint64_t(a.B * a.S)};
+    const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hkv) * HD * 2};
+    const uint32_t box[3] = {64, 1, uint32_t(Cfg::BK)};
+    if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+    if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+  }
+  FwdParams p;
+  p.units = a.units;
+  p.n_units = a.n_units;
+  p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.S = a.S;
+  p.C = a.S / (2 * int64_t(a.D));
+  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.D = a.D; p.causal = a.causal;
+  p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
+  p.status = a.status;
+  p.wait_limit_ns = a.wait_limit_ns;
+  p.inject_stall = a.inject_stall;
+  const int smem = Cfg::SMEM_BYTES + 1024;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(zsa_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return int(e);
+    attr_set = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = a.n_units < sms ? a.n_units : sms;
+  if (grid <= 0) return int(cudaSuccess);
+  zsa_fwd_kernel<HD><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, p);
+  return int(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_fwd(const FwdArgs& a, cudaStream_t stream) {
+  switch (a.d) {
+    case 64: return launch_fwd_hd<64>(a, stream);
+    case 128: return launch_fwd_hd<128>(a, stream);
+    case 256: return launch_fwd_hd<256>(a, stream);
+    default: return int(cudaErrorInvalidValue);
+  }
+}
+
+}  // namespace zsa

@@ -1,0 +1,57 @@
+// zsa_kernels.h -- host-side launch interface of the sm_100a kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "zsa_schedule.h"
+
+namespace zsa {
+
+struct FwdArgs {
+  const void* q;           // [D][B][2C][Hq][d] bf16
+  const void* k;           // [B][S][Hkv][d] bf16
+  const void* v;
+  void* o;                 // [D][B][2C][Hq][d] bf16
+  float* lse;              // [D][B][Hq][2C]
+  const DevUnit* units;    // device copy of the schedule
+  int32_t n_units;
+  int64_t S;
+  int32_t B, Hq, Hkv, d, D, causal;
+  float scale;
+  int* status;
+  uint64_t wait_limit_ns;
+  int inject_stall;        // test hook: MMA thread first waits on a barrier nobody arrives at
+};
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const float* lse;
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* delta;            // [D][B][Hq][2C] workspace
+  float* dq_acc;           // [D][B][2C][Hq][d] workspace
+  int64_t S;
+  int32_t B, Hq, Hkv, d, D, causal;
+  float scale;
+  int* status;
+  uint64_t wait_limit_ns;
+  int inject_stall;        // test hook: MMA thread first waits on a barrier nobody arrives at
+};
+
+// Tiling the forward kernel is built for, per head dim.
+inline void fwd_tiling(int d, int32_t* bq, int32_t* bk, int32_t* slots) {
+  *bq = 128;
+  *bk = d <= 128 ? 128 : 64;
+  *slots = d <= 128 ? 2 : 1;
+}
+
+// Returns a cudaError_t (cudaSuccess on success).
+int launch_fwd(const FwdArgs& a, cudaStream_t stream);
+int launch_bwd(const BwdArgs& a, cudaStream_t stream);
+
+}  // namespace zsa

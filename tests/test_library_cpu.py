@@ -1,0 +1,106 @@
+"""Host-side checks of libzsa that need no GPU.
+
+- the library loads and exports every entry point include/zsa.h declares;
+- zsa_partition (zigzag map, per-shard tile work, unit schedule) equals the oracle's
+  independently written partition and schedule, bit for bit, over a sweep of shapes
+  and tilings including the five benchmark configurations;
+- argument errors come back as the documented status codes before anything touches
+  a device.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import sequence_sharded_causal_b200 as zsa
+from sequence_sharded_causal_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return zsa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    header = open(os.path.join(ROOT, "include", "zsa.h")).read()
+    declared = set(re.findall(r"^\s*ZSA_API\s+(?:int|const char\*)\s+(zsa_\w+)\s*\(", header, re.M))
+    assert declared == set(zsa.EXPORTED), declared
+    for name in declared:
+        assert hasattr(L, name), name
+    assert zsa.status_string(zsa.ZSA_ERR_TIMEOUT).startswith("a bounded")
+
+
+CONFIGS = [  # (B, S, Hq, Hkv, d, D): the five benchmark shapes
+    (1, 256, 2, 2, 64, 2), (1, 16384, 32, 32, 128, 8), (1, 32768, 32, 8, 128, 8),
+    (1, 65536, 24, 4, 256, 4), (1, 131072, 32, 8, 128, 16)]
+
+
+@pytest.mark.parametrize("cfg", CONFIGS)
+def test_partition_matches_oracle_on_configs(L, oracle, cfg):
+    B, S, Hq, Hkv, d, D = cfg
+    p = zsa.make_problem(B, S, Hq, Hkv, d, D)
+    got = zsa.zsa_partition(p)
+    perm, inv = oracle.partition(S, D)
+    assert np.array_equal(got["perm"], perm)
+    assert np.array_equal(got["inv_perm"], inv)
+    bq, bk, slots = got["tiling"]
+    st, units = oracle.schedule(S, D, B, Hq, Hkv, True, bq, bk, slots)
+    assert np.array_equal(got["shard_tiles"], st)
+    assert np.array_equal(got["sched"], units)
+    assert len(set(got["shard_tiles"].tolist())) == 1
+
+
+SWEEP = [(S, D, B, Hq, Hkv, bq, bk, slots, causal)
+         for (S, D) in ((256, 2), (512, 1), (768, 2), (1536, 4), (2560, 5), (4096, 8))
+         for (B, Hq, Hkv) in ((1, 2, 2), (2, 6, 2), (1, 3, 1), (1, 8, 8))
+         for (bq, bk) in ((128, 128), (128, 64), (64, 64))
+         for slots in (1, 2) for causal in (0, 1)
+         if (S // D) % bq == 0]
+
+
+@pytest.mark.parametrize("S,D,B,Hq,Hkv,bq,bk,slots,causal", SWEEP[::3])
+def test_schedule_sweep_bit_exact(L, oracle, S, D, B, Hq, Hkv, bq, bk, slots, causal):
+    p = zsa.make_problem(B, S, Hq, Hkv, 128, D, causal)
+    got = zsa.zsa_partition(p, bq, bk, slots)
+    st, units = oracle.schedule(S, D, B, Hq, Hkv, bool(causal), bq, bk, slots)
+    assert np.array_equal(got["shard_tiles"], st)
+    assert np.array_equal(got["sched"], units)
+
+
+def _rc_fwd(L, problem, ptrs=(16,) * 5, ws=256, ws_bytes=1 << 30):
+    return L.zsa_attn_fwd(ctypes.byref(problem), *ptrs, ws, ws_bytes, None)
+
+
+def test_argument_errors(L):
+    good = zsa.make_problem(1, 1024, 4, 2, 128, 2)
+    assert _rc_fwd(L, good, ptrs=(None, 16, 16, 16, 16)) == zsa.ZSA_ERR_INVALID
+    assert _rc_fwd(L, good, ptrs=(24, 16, 16, 16, 16)) == zsa.ZSA_ERR_INVALID   # misaligned
+    assert _rc_fwd(L, good, ws=272) == zsa.ZSA_ERR_INVALID                        # ws not 256-aligned
+    assert _rc_fwd(L, zsa.make_problem(1, 1024, 4, 3, 128, 2)) == zsa.ZSA_ERR_SHAPE   # Hq % Hkv
+    assert _rc_fwd(L, zsa.make_problem(1, 1000, 4, 2, 128, 2)) == zsa.ZSA_ERR_SHAPE   # S % 2D*64
+    assert _rc_fwd(L, zsa.make_problem(1, 768, 4, 2, 128, 4)) == zsa.ZSA_ERR_SHAPE
+    assert _rc_fwd(L, zsa.make_problem(1, 1024, 4, 2, 96, 2)) == zsa.ZSA_ERR_UNSUPPORTED
+    assert _rc_fwd(L, zsa.make_problem(0, 1024, 4, 2, 128, 2)) == zsa.ZSA_ERR_INVALID
+    assert _rc_fwd(L, zsa.make_problem(1, 1024, 4, 2, 128, 2, scale=-1.0)) == zsa.ZSA_ERR_INVALID
+    assert _rc_fwd(L, good, ws_bytes=64) == zsa.ZSA_ERR_WORKSPACE
+    assert L.zsa_attn_fwd(None, 16, 16, 16, 16, 16, 256, 1 << 30, None) == zsa.ZSA_ERR_INVALID
+    bw = [16] * 9
+    assert L.zsa_attn_bwd(ctypes.byref(good), *bw, 256, 64, None) == zsa.ZSA_ERR_WORKSPACE
+    bw[3] = None
+    assert L.zsa_attn_bwd(ctypes.byref(good), *bw, 256, 1 << 40, None) == zsa.ZSA_ERR_INVALID
+    out = ctypes.c_size_t(0)
+    assert L.zsa_workspace_bytes(ctypes.byref(good), 2, ctypes.byref(out)) == zsa.ZSA_ERR_INVALID
+    assert L.zsa_workspace_bytes(ctypes.byref(good), 1, ctypes.byref(out)) == zsa.ZSA_OK
+    assert out.value >= 1024 * 4 * (128 + 1) * 4
+    n = ctypes.c_int64(0)
+    t = zsa.zsa_tiling(0, 0, 0)
+    sched = (zsa.zsa_work * 1)()
+    rc = L.zsa_partition(ctypes.byref(good), ctypes.byref(t), None, None, None,
+                         ctypes.cast(sched, ctypes.c_void_p), 1, ctypes.byref(n))
+    assert rc == zsa.ZSA_ERR_WORKSPACE and n.value > 1
+    assert (t.block_q, t.block_k, t.slots) == (128, 128, 2)
