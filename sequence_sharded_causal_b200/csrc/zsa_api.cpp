@@ -266,6 +266,7 @@ int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t stats = size_t(problem->B) * problem->S * problem->Hq * sizeof(float);
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return ZSA_ERR_CUDA;
   zsa::BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
   a.dq = dq; a.dk = dk; a.dv = dv;

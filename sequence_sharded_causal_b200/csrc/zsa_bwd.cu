@@ -1,8 +1,733 @@
-// zsa_bwd.cu -- backward kernels (K2 preprocess, K3 main, K4 dQ epilogue).
+// zsa_bwd.cu -- backward of zigzag-sharded causal GQA attention on sm_100a.
+//
+// The pages describe only the forward (all-gathered K/V + FlashAttention with a zigzag
+// partition, "Folding Tensor and Sequence Parallelism" summary, section 2); the
+// backward here is the exact gradient of <dO, O>, recomputing P from the saved lse:
+//   Delta = rowsum(dO * O)                                            (K2, HBM-bound)
+//   per key tile (b, kv head g, n), over every (shard, q tile, q head of g) that sees it:
+//     S^T = K Q^T,  P^T = exp(scale S^T - lse),  dP^T = V dO^T,
+//     dS^T = P^T * (dP^T - Delta),
+//     dV += P^T dO,  dK += dS^T Q,  dQ^T (+)= K^T dS^T                 (K3, tensor-bound)
+//   dQ = bf16(scale * dQacc)                                          (K4, HBM-bound)
+// dK and dV are summed over every shard and the G q heads of the group inside one CTA
+// (the single-GPU stand-in for the reduce-scatter back to the owning shards); dQ is
+// summed across key tiles with fp32 reductions into a workspace accumulator.
+//
+// K3 layout (d = 128; d = 64 uses the same code with half-width accumulators):
+//  * one persistent CTA per SM walks key tiles (n ascending = most work first; snake
+//    order over CTAs); K and V (128 keys) stay in shared memory for the whole tile;
+//  * q slots are 64-row tiles (a 64-row tile never straddles a zigzag chunk because
+//    C is a multiple of 64) streamed through a 2-stage ring: Q, dO, lse, Delta;
+//  * TMEM: dV | dK (fp32, 128 lanes = keys) | S^T x2 | dP^T | dQ^T (64 cols each);
+//    P^T and dS^T are written back as bf16 over the columns they came from and feed
+//    the dV / dK MMAs as TMEM A operands; dS^T also goes to shared memory (128B
+//    swizzle) as the MN-major B operand of dQ^T = K^T dS^T, whose A operand is the
+//    resident K tile read as an MN-major (transposed) operand;
+//  * warps: 8 compute warps (two groups split each slot's 64 columns), 4 dQ warps
+//    (TMEM -> fp32 reductions into the dQ accumulator), 1 TMA producer, 1 MMA issuer.
+#include <cuda_bf16.h>
+
 #include "zsa_kernels.h"
+#include "zsa_ptx.cuh"
+#include "zsa_tma_host.h"
 
 namespace zsa {
+namespace {
 
-int launch_bwd(const BwdArgs&, cudaStream_t) { return int(cudaErrorNotSupported); }
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ K2: Delta + zero dQacc
+template <int HD>
+__global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                          const __nv_bfloat16* __restrict__ dout,
+                                                          float* __restrict__ delta,
+                                                          float* __restrict__ dq_acc,
+                                                          int64_t n_pairs, int32_t Hq,
+                                                          int64_t twoC) {
+  constexpr int LPP = HD / 8;  // lanes per (row, head) pair, 8 bf16 (16 B) per lane
+  const int lane = int(threadIdx.x & 31);
+  const int sub = lane % LPP;
+  const int64_t warp_global = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int64_t n_warps = int64_t(gridDim.x) * blockDim.x / 32;
+  for (int64_t base = warp_global * (32 / LPP); base < n_pairs; base += n_warps * (32 / LPP)) {
+    const int64_t pair = base + lane / LPP;
+    float acc = 0.f;
+    if (pair < n_pairs) {
+      const uint4 a = reinterpret_cast<const uint4*>(o + pair * HD)[sub];
+      const uint4 b = reinterpret_cast<const uint4*>(dout + pair * HD)[sub];
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 x = __bfloat1622float2(a2[t]);
+        const float2 y = __bfloat1622float2(b2[t]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+      float4* z = reinterpret_cast<float4*>(dq_acc + pair * HD) + 2 * sub;
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = LPP / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (pair < n_pairs && sub == 0) {
+      const int64_t row = pair / Hq;           // (r*B + b)*2C + j
+      const int32_t h = int32_t(pair % Hq);
+      const int64_t rb = row / twoC, j = row % twoC;
+      delta[(rb * Hq + h) * twoC + j] = acc;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ K4: dQ = bf16(scale*acc)
+__global__ void __launch_bounds__(256) zsa_dq_convert_kernel(const float* __restrict__ acc,
+                                                             __nv_bfloat16* __restrict__ dq,
+                                                             int64_t n8, float scale) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    uint4 r;
+    r.x = pack_bf16x2(a.x * scale, a.y * scale);
+    r.y = pack_bf16x2(a.z * scale, a.w * scale);
+    r.z = pack_bf16x2(b.x * scale, b.y * scale);
+    r.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[i] = r;
+  }
+}
+
+// ------------------------------------------------------------------ K3: main backward
+template <int HD>
+struct BwdCfg {
+  static constexpr int BKV = 128;   // keys per CTA tile (TMEM lanes)
+  static constexpr int BQ = 64;     // query rows per slot
+  static constexpr int KB = HD / 64;
+  static constexpr int NQST = 2;    // Q/dO stages
+  static constexpr int KV_BYTES = BKV * HD * 2;          // K (or V) tile
+  static constexpr int QT_BYTES = BQ * HD * 2;           // Q (or dO) slot tile
+  static constexpr int DS_BYTES = BKV * BQ * 2;          // dS^T tile (bf16)
+  static constexpr int SMEM_K = 0;
+  static constexpr int SMEM_V = SMEM_K + KV_BYTES;
+  static constexpr int SMEM_Q = SMEM_V + KV_BYTES;
+  static constexpr int SMEM_DO = SMEM_Q + NQST * QT_BYTES;
+  static constexpr int SMEM_DS = SMEM_DO + NQST * QT_BYTES;
+  static constexpr int SMEM_LSE = SMEM_DS + 2 * DS_BYTES;      // [NQST][BQ] fp32
+  static constexpr int SMEM_DELTA = SMEM_LSE + NQST * BQ * 4;  // [NQST][BQ] fp32
+  static constexpr int SMEM_BYTES = SMEM_DELTA + NQST * BQ * 4;
+  static constexpr int WARP_DQ = 8;       // warps 8..11
+  static constexpr int WARP_LOAD = 12;
+  static constexpr int WARP_MMA = 13;
+  static constexpr int NTHREADS = 14 * 32;
+  static constexpr uint32_t TM_DV = 0;
+  static constexpr uint32_t TM_DK = HD;
+  static constexpr uint32_t TM_ST = 2 * HD;        // two buffers of 64 columns
+  static constexpr uint32_t TM_DPT = 2 * HD + 128;
+  static constexpr uint32_t TM_DQT = 2 * HD + 192;
+  static constexpr uint32_t TM_COLS = 512;
+  static_assert(2 * HD + 256 <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
+};
+
+struct BwdParams {
+  const float* lse;
+  const float* delta;
+  float* dq_acc;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int64_t S, C;
+  int32_t B, Hq, Hkv, G, D, causal;
+  int32_t n_units, n_qtiles;  // n_qtiles = 64-row tiles per shard
+  float scale, scale_log2;
+  int* status;
+  uint64_t wait_limit_ns;
+  int inject_stall;
+};
+
+struct BwdBars {
+  uint64_t kv_full, kv_empty;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], st_free[2];
+  uint64_t dp_full, dpt_free;
+  uint64_t p_full, ds_full;
+  uint64_t dsm_free[2];
+  uint64_t dq_full, dq_empty;
+  uint64_t acc_full, acc_empty;
+  uint64_t drain, never;
+};
+
+// One key tile of work.
+struct KvUnit {
+  int32_t n, b, g;
+};
+
+__device__ __forceinline__ int bwd_unit_index(int k, int n_units) {
+  const int grid = int(gridDim.x);
+  const int idx = k * grid + ((k & 1) ? (grid - 1 - int(blockIdx.x)) : int(blockIdx.x));
+  return idx < n_units ? idx : -1;
+}
+
+__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int B, int Hkv) {
+  KvUnit u;
+  u.n = idx / (B * Hkv);
+  const int rem = idx % (B * Hkv);
+  u.b = rem / Hkv;
+  u.g = rem % Hkv;
+  return u;
+}
+
+// Enumerates the q slots (shard r, 64-row tile i, head offset e) that see key tile n,
+// in (r, i, e) order.  Every role walks the same sequence.
+struct SlotWalk {
+  int32_t r, i, e;
+  int64_t p0;   // position of the tile's first row (its rows are p0 .. p0+63)
+};
+
+__device__ __forceinline__ int64_t zz_pos(int64_t C, int32_t D, int32_t r, int64_t j) {
+  return j < C ? int64_t(r) * C + j : int64_t(2 * D - 1 - r) * C + (j - C);
+}
+
+__device__ __forceinline__ bool tile_sees(const BwdParams& p, int32_t r, int32_t i, int32_t n,
+                                          int64_t* p0) {
+  *p0 = zz_pos(p.C, p.D, r, int64_t(i) * 64);
+  return !p.causal || (*p0 + 63 >= int64_t(n) * 128);
+}
+
+// First slot at or after (r, i, 0); false when the walk is over.
+__device__ __forceinline__ bool walk_seek(const BwdParams& p, int32_t n, SlotWalk& w) {
+  while (w.r < p.D) {
+    if (tile_sees(p, w.r, w.i, n, &w.p0)) return true;
+    if (++w.i == p.n_qtiles) {
+      w.i = 0;
+      ++w.r;
+    }
+  }
+  return false;
+}
+__device__ __forceinline__ bool walk_first(const BwdParams& p, int32_t n, SlotWalk& w) {
+  w.r = 0; w.i = 0; w.e = 0;
+  return walk_seek(p, n, w);
+}
+__device__ __forceinline__ bool walk_next(const BwdParams& p, int32_t n, SlotWalk& w) {
+  if (++w.e < p.G) return true;
+  w.e = 0;
+  if (++w.i == p.n_qtiles) {
+    w.i = 0;
+    ++w.r;
+  }
+  return walk_seek(p, n, w);
+}
+
+__device__ __forceinline__ bool warp_wait_b(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  bool ok = mbar_wait(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
+    zsa_bwd_kernel(const __grid_constant__ CUtensorMap map_q,
+                   const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v,
+                   const __grid_constant__ CUtensorMap map_do, const BwdParams prm) {
+  using Cfg = BwdCfg<HD>;
+  constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ BwdBars bars;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  const int warp = int(warp_id()), lane = int(lane_id());
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    mbar_init(&bars.kv_full, 1);
+    mbar_init(&bars.kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_empty[s], 1 + 8);   // MMA commit + 8 compute warps
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.st_free[s], 1);
+      mbar_init(&bars.dsm_free[s], 1);
+    }
+    mbar_init(&bars.dp_full, 1);
+    mbar_init(&bars.dpt_free, 1);
+    mbar_init(&bars.p_full, 8);
+    mbar_init(&bars.ds_full, 8);
+    mbar_init(&bars.dq_full, 1);
+    mbar_init(&bars.dq_empty, 4);
+    mbar_init(&bars.acc_full, 1);
+    mbar_init(&bars.acc_empty, 8);
+    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.never, 1);
+    fence_mbar_init();
+  }
+  if (warp == Cfg::WARP_MMA) {
+    tmem_alloc(&tmem_base_s, Cfg::TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == Cfg::WARP_LOAD && lane == 0) {
+    tma_prefetch_desc(&map_q);
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_v);
+    tma_prefetch_desc(&map_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  const WaitCtx wctx{&abort_s, prm.status, prm.wait_limit_ns};
+  const int64_t twoC = 2 * prm.C;
+
+  if (warp == Cfg::WARP_LOAD) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t q_it = 0, kv_fills = 0;
+      uint32_t q_fills[2] = {0, 0};
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int idx = bwd_unit_index(k, prm.n_units);
+        if (idx < 0) break;
+        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+        if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
+        if (!ok) break;
+        mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
+        const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(u.n) * BKV);
+        for (int kb = 0; kb < KB; ++kb) {
+          tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128, &map_k, &bars.kv_full, kb * 64, u.g, key0);
+          tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128, &map_v, &bars.kv_full, kb * 64, u.g, key0);
+        }
+        ++kv_fills;
+        SlotWalk w;
+        for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
+          const int st = int(q_it & 1);
+          const uint32_t use = q_it >> 1;
+          if (use > 0) ok = mbar_wait(&bars.q_empty[st], (use - 1) & 1, wctx);
+          if (!ok) break;
+          const int32_t h = u.g * prm.G + w.e;
+          const int64_t rb = int64_t(w.r) * prm.B + u.b;
+          const int32_t row0 = int32_t(rb * twoC + int64_t(w.i) * BQ);
+          mbar_expect_tx(&bars.q_full[st], 2 * Cfg::QT_BYTES + 2 * BQ * 4);
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d(smem + Cfg::SMEM_Q + st * Cfg::QT_BYTES + kb * BQ * 128, &map_q,
+                        &bars.q_full[st], kb * 64, h, row0);
+            tma_load_3d(smem + Cfg::SMEM_DO + st * Cfg::QT_BYTES + kb * BQ * 128, &map_do,
+                        &bars.q_full[st], kb * 64, h, row0);
+          }
+          const int64_t stat = (rb * prm.Hq + h) * twoC + int64_t(w.i) * BQ;
+          bulk_load(smem + Cfg::SMEM_LSE + st * BQ * 4, prm.lse + stat, BQ * 4, &bars.q_full[st]);
+          bulk_load(smem + Cfg::SMEM_DELTA + st * BQ * 4, prm.delta + stat, BQ * 4, &bars.q_full[st]);
+          ++q_fills[st];
+          ++q_it;
+        }
+      }
+      if (!ok) {
+        const uint64_t lim = 1000000000ull;
+        if (kv_fills > 0) mbar_drain(&bars.kv_full, (kv_fills - 1) & 1, lim);
+        for (int s = 0; s < 2; ++s)
+          if (q_fills[s] > 0) mbar_drain(&bars.q_full[s], (q_fills[s] - 1) & 1, lim);
+      }
+    }
+  } else if (warp == Cfg::WARP_MMA) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(128, BQ, false, false);
+      const uint32_t idesc_kv = idesc_bf16(128, HD, false, true);
+      const uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);
+      const uint32_t sK = smem_u32(smem + Cfg::SMEM_K);
+      const uint32_t sV = smem_u32(smem + Cfg::SMEM_V);
+      const uint32_t sQ = smem_u32(smem + Cfg::SMEM_Q);
+      const uint32_t sDO = smem_u32(smem + Cfg::SMEM_DO);
+      const uint32_t sDS = smem_u32(smem + Cfg::SMEM_DS);
+      // dQ^T = K^T dS^T: A = K^T, M = d in 64-row blocks at the d-block stride of the K
+      // tile.  With d = 64 the second M block points at V (its rows are never read).
+      const uint32_t lbo_kt = HD >= 128 ? uint32_t(BKV * 128) : uint32_t(Cfg::SMEM_V - Cfg::SMEM_K);
+      uint32_t kv_ph = 0, q_it = 0;
+      uint32_t q_full_uses[2] = {0, 0};
+      uint32_t p_ph = 0, ds_ph = 0;
+      uint32_t st_commits[2] = {0, 0}, st_waits[2] = {0, 0};
+      uint32_t dpt_commits = 0, dpt_waits = 0;
+      uint32_t dq_commits = 0, dq_waits = 0;
+      uint32_t acc_commits = 0;
+      bool ok = true;
+      if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
+      auto wait_st_free = [&](int b) {
+        if (st_commits[b] > st_waits[b]) {
+          ok = ok && mbar_wait(&bars.st_free[b], st_waits[b] & 1, wctx);
+          ++st_waits[b];
+        }
+      };
+      auto wait_dpt_free = [&]() {
+        if (dpt_commits > dpt_waits) {
+          ok = ok && mbar_wait(&bars.dpt_free, dpt_waits & 1, wctx);
+          ++dpt_waits;
+        }
+      };
+      auto issue_st = [&](int st, int b) {       // S^T = K Q^T
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + Cfg::TM_ST + b * 64, sdesc_sw128(sK + kb * BKV * 128 + ks * 32, 16, 1024),
+                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
+                   idesc_s, (kb | ks) != 0);
+      };
+      auto issue_dpt = [&](int st) {             // dP^T = V dO^T
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + Cfg::TM_DPT, sdesc_sw128(sV + kb * BKV * 128 + ks * 32, 16, 1024),
+                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
+                   idesc_s, (kb | ks) != 0);
+      };
+      for (int k = 0; ok; ++k) {
+        const int idx = bwd_unit_index(k, prm.n_units);
+        if (idx < 0) break;
+        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+        ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
+        kv_ph ^= 1;
+        if (!ok) break;
+        SlotWalk w;
+        bool more = walk_first(prm, u.n, w);
+        // prologue: S^T(0), dP^T(0)
+        if (more) {
+          const int st = int(q_it & 1);
+          ok = mbar_wait(&bars.q_full[st], q_full_uses[st] & 1, wctx);
+          ++q_full_uses[st];
+          wait_st_free(0);
+          if (!ok) break;
+          tc_fence_after();
+          issue_st(st, 0);
+          mma_commit(&bars.s_full[0]);
+          wait_dpt_free();
+          if (!ok) break;
+          tc_fence_after();
+          issue_dpt(st);
+          mma_commit(&bars.dp_full);
+        }
+        for (int j = 0; more && ok; ++j) {
+          const int b = j & 1;
+          const int st = int(q_it & 1);
+          SlotWalk nx = w;
+          const bool has_next = walk_next(prm, u.n, nx);
+          const int st1 = int((q_it + 1) & 1);
+          // dV += P^T dO
+          ok = mbar_wait(&bars.p_full, p_ph, wctx);
+          p_ph ^= 1;
+          if (ok && j == 0 && acc_commits > 0)
+            ok = mbar_wait(&bars.acc_empty, (acc_commits - 1) & 1, wctx);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BQ / 16; ++ks)
+            mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + b * 64 + (ks >> 1) * 32 + (ks & 1) * 8,
+                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+                   (j > 0) || (ks > 0));
+          mma_commit(&bars.st_free[b]);
+          ++st_commits[b];
+          // next slot's S^T into the other buffer
+          if (has_next) {
+            ok = mbar_wait(&bars.q_full[st1], q_full_uses[st1] & 1, wctx);
+            ++q_full_uses[st1];
+            wait_st_free(b ^ 1);
+            if (!ok) break;
+            tc_fence_after();
+            issue_st(st1, b ^ 1);
+            mma_commit(&bars.s_full[b ^ 1]);
+          }
+          // dK += dS^T Q ; dQ^T = K^T dS^T
+          ok = mbar_wait(&bars.ds_full, ds_ph, wctx);
+          ds_ph ^= 1;
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BQ / 16; ++ks)
+            mma_ts(tmem + Cfg::TM_DK, tmem + Cfg::TM_DPT + (ks >> 1) * 32 + (ks & 1) * 8,
+                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+                   (j > 0) || (ks > 0));
+          mma_commit(&bars.dpt_free);
+          ++dpt_commits;
+          if (dq_commits > dq_waits) {
+            ok = mbar_wait(&bars.dq_empty, dq_waits & 1, wctx);
+            ++dq_waits;
+            if (!ok) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int ks = 0; ks < BKV / 16; ++ks)
+            mma_ss(tmem + Cfg::TM_DQT, sdesc_sw128(sK + ks * 2048, lbo_kt, 1024),
+                   sdesc_sw128(sDS + b * Cfg::DS_BYTES + ks * 2048, BQ * 128, 1024), idesc_dq,
+                   ks > 0);
+          mma_commit(&bars.dq_full);
+          ++dq_commits;
+          mma_commit(&bars.dsm_free[b]);
+          mma_commit(&bars.q_empty[st]);
+          ++q_it;
+          // next slot's dP^T once dK has consumed dS^T from the dP^T columns
+          if (has_next) {
+            wait_dpt_free();
+            if (!ok) break;
+            tc_fence_after();
+            issue_dpt(st1);
+            mma_commit(&bars.dp_full);
+          }
+          w = nx;
+          more = has_next;
+        }
+        if (!ok) break;
+        mma_commit(&bars.acc_full);
+        ++acc_commits;
+        mma_commit(&bars.kv_empty);
+      }
+      mma_commit(&bars.drain);
+      mbar_drain(&bars.drain, 0, 1000000000ull);
+    }
+    __syncwarp();
+  } else if (warp >= Cfg::WARP_DQ) {
+    // ------------------------------------------------------------ dQ warps
+    const int qw = warp - Cfg::WARP_DQ;
+    const int drow = qw * 32 + lane;           // TMEM lane = d index of dQ^T
+    const uint32_t tDQ = tmem + Cfg::TM_DQT + (uint32_t(qw * 32) << 16);
+    uint32_t dq_ph = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = bwd_unit_index(k, prm.n_units);
+      if (idx < 0) break;
+      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+      SlotWalk w;
+      for (bool more = walk_first(prm, u.n, w); more; more = walk_next(prm, u.n, w)) {
+        ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
+        dq_ph ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tDQ, v0);
+        tmem_ld32(tDQ + 32, v1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.dq_empty);
+        if (drow < HD) {
+          const int32_t h = u.g * prm.G + w.e;
+          const int64_t row0 = (int64_t(w.r) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
+          float* base = prm.dq_acc + (row0 * prm.Hq + h) * HD + drow;
+          const int64_t rstride = int64_t(prm.Hq) * HD;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) atomicAdd(base + c * rstride, __uint_as_float(v0[c]));
+#pragma unroll
+          for (int c = 0; c < 32; ++c) atomicAdd(base + (32 + c) * rstride, __uint_as_float(v1[c]));
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ compute warps
+    const int half = warp / 4;                 // which 32 of the slot's 64 columns
+    const int qw = warp % 4;
+    const int row = qw * 32 + lane;            // TMEM lane = key within the tile
+    const uint32_t lane_addr = uint32_t(qw * 32) << 16;
+    const float* sLse = reinterpret_cast<const float*>(smem + Cfg::SMEM_LSE);
+    const float* sDelta = reinterpret_cast<const float*>(smem + Cfg::SMEM_DELTA);
+    uint8_t* sDS = smem + Cfg::SMEM_DS;
+    uint32_t q_it = 0, q_full_uses[2] = {0, 0};
+    uint32_t s_ph[2] = {0, 0}, dp_ph = 0, acc_ph = 0;
+    uint32_t dsm_uses[2] = {0, 0};
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = bwd_unit_index(k, prm.n_units);
+      if (idx < 0) break;
+      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+      const int64_t key = int64_t(u.n) * BKV + row;
+      SlotWalk w;
+      int j = 0;
+      for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w), ++j) {
+        const int b = j & 1;
+        const int st = int(q_it & 1);
+        ok = warp_wait_b(&bars.q_full[st], q_full_uses[st] & 1, wctx);
+        ++q_full_uses[st];
+        if (!ok) break;
+        // per-column statistics of this warp's 32 query rows, read from shared memory
+        const float* lse_c = sLse + st * BQ + half * 32;
+        const float* dlt_c = sDelta + st * BQ + half * 32;
+        // causal mask: column c holds position p0 + half*32 + c; masked when key > it
+        const int64_t first = w.p0 + half * 32;
+        const int nvis_lo = prm.causal ? int(key - first) : 0;   // columns c < nvis_lo are masked
+        // ---- P^T
+        ok = warp_wait_b(&bars.s_full[b], s_ph[b], wctx);
+        s_ph[b] ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sv[32];
+        tmem_ld32(tmem + Cfg::TM_ST + b * 64 + half * 32 + lane_addr, sv);
+        tmem_ld_wait();
+        float pf[32];
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float x = fmaf(__uint_as_float(sv[c]), prm.scale_log2, -lse_c[c] * kLog2e);
+          pf[c] = (c < nvis_lo) ? 0.f : ex2_approx(x);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
+        tmem_st16(tmem + Cfg::TM_ST + b * 64 + half * 32 + lane_addr, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full);
+        // ---- dS^T
+        ok = warp_wait_b(&bars.dp_full, dp_ph, wctx);
+        dp_ph ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        tmem_ld32(tmem + Cfg::TM_DPT + half * 32 + lane_addr, sv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(pf[2 * e] * (__uint_as_float(sv[2 * e]) - dlt_c[2 * e]),
+                              pf[2 * e + 1] * (__uint_as_float(sv[2 * e + 1]) - dlt_c[2 * e + 1]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.q_empty[st]);   // lse / Delta of this stage consumed
+        ++q_it;
+        tmem_st16(tmem + Cfg::TM_DPT + half * 32 + lane_addr, pk);
+        // shared-memory copy for dQ^T: row = key, 16-byte chunks 4*half .. 4*half+3
+        if (dsm_uses[b] > 0) {
+          ok = warp_wait_b(&bars.dsm_free[b], (dsm_uses[b] - 1) & 1, wctx);
+          if (!ok) break;
+        }
+        ++dsm_uses[b];
+        uint8_t* dsb = sDS + b * Cfg::DS_BYTES;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4*>(dsb + sw128_offset(uint32_t(row), uint32_t(4 * half + m))) =
+              make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.ds_full);
+      }
+      if (!ok) break;
+      // ---- epilogue: dV (first group) / dK (second group) rows of this key tile
+      ok = warp_wait_b(&bars.acc_full, acc_ph, wctx);
+      acc_ph ^= 1;
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tAcc = tmem + (half == 0 ? Cfg::TM_DV : Cfg::TM_DK) + lane_addr;
+      const float mul = half == 0 ? 1.0f : prm.scale;
+      __nv_bfloat16* dst = (half == 0 ? prm.dv : prm.dk) +
+                           ((int64_t(u.b) * prm.S + key) * prm.Hkv + u.g) * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tAcc + c * 32, a);
+        tmem_ld_wait();
+        uint32_t o16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          o16[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * mul, __uint_as_float(a[2 * e + 1]) * mul);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          d4[v4] = make_uint4(o16[4 * v4], o16[4 * v4 + 1], o16[4 * v4 + 2], o16[4 * v4 + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == Cfg::WARP_MMA) tmem_dealloc(tmem, Cfg::TM_COLS);
+}
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <int HD>
+int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
+  using Cfg = BwdCfg<HD>;
+  const int64_t rows = a.S * a.B;             // shard-major rows (D * B * 2C)
+  const int64_t twoC = a.S / a.D;
+  const int sms = num_sms();
+  // K2: Delta and a zeroed dQ accumulator
+  {
+    const int64_t pairs = rows * a.Hq;
+    const int64_t warps_needed = (pairs + (256 / HD) * 4 - 1) / ((256 / HD) * 4);
+    int64_t blocks = (warps_needed + 7) / 8;
+    if (blocks > int64_t(sms) * 16) blocks = int64_t(sms) * 16;
+    if (blocks < 1) blocks = 1;
+    zsa_bwd_pre_kernel<HD><<<int(blocks), 256, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16*>(a.o), reinterpret_cast<const __nv_bfloat16*>(a.dout),
+        a.delta, a.dq_acc, pairs, a.Hq, twoC);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return int(e);
+  }
+  // K3
+  CUtensorMap mq, mk, mv, mdo;
+  {
+    const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hq), uint64_t(rows)};
+    const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hq) * HD * 2};
+    const uint32_t box[3] = {64, 1, uint32_t(Cfg::BQ)};
+    if (!make_map_bf16_sw128(&mq, a.q, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+    if (!make_map_bf16_sw128(&mdo, a.dout, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+  }
+  {
+    const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), uint64_t(a.B * a.S)};
+    const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hkv) * HD * 2};
+    const uint32_t box[3] = {64, 1, uint32_t(Cfg::BKV)};
+    if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+    if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+  }
+  BwdParams p;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.dq_acc = a.dq_acc;
+  p.dk = reinterpret_cast<__nv_bfloat16*>(a.dk);
+  p.dv = reinterpret_cast<__nv_bfloat16*>(a.dv);
+  p.S = a.S;
+  p.C = a.S / (2 * int64_t(a.D));
+  p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = a.Hq / a.Hkv; p.D = a.D; p.causal = a.causal;
+  p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / Cfg::BKV));
+  p.n_qtiles = int32_t(twoC / Cfg::BQ);
+  p.scale = a.scale;
+  p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
+  p.status = a.status;
+  p.wait_limit_ns = a.wait_limit_ns;
+  p.inject_stall = a.inject_stall;
+  const int smem = Cfg::SMEM_BYTES + 1024;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(zsa_bwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return int(e);
+    attr_set = true;
+  }
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  zsa_bwd_kernel<HD><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return int(e);
+  // K4
+  {
+    const int64_t n8 = rows * a.Hq * HD / 8;
+    int64_t blocks = (n8 + 255) / 256;
+    if (blocks > int64_t(sms) * 16) blocks = int64_t(sms) * 16;
+    zsa_dq_convert_kernel<<<int(blocks), 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq),
+                                                            n8, a.scale);
+    e = cudaGetLastError();
+  }
+  return int(e);
+}
+
+}  // namespace
+
+int launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  switch (a.d) {
+    case 64: return launch_bwd_hd<64>(a, stream);
+    case 128: return launch_bwd_hd<128>(a, stream);
+    default: return int(cudaErrorNotSupported);
+  }
+}
 
 }  // namespace zsa
