@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Benchmark: zigzag-sharded causal attention, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl zsa|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input: the
+forward (zsa_attn_fwd: zigzag schedule + forward kernel) and the backward
+(zsa_attn_bwd: Delta preprocess, backward main kernel, dQ conversion), all D logical
+shards in one launch each.  Throughput is algorithmic causal FLOPs per second:
+forward 4*B*Hq*d*S(S+1)/2, backward 2.5x that.
+
+--gpus N > 1 runs N independent replicas (the single-GPU path has no collective;
+launch with torchrun); value is the sum over ranks, time the max over ranks.
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
+Prints ONE JSON line on rank 0.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "causal attn fwd+bwd TFLOP/s at 1 B200 and % of BF16 tensor peak"
+L2_BYTES = 126 * 2**20
+
+CONFIGS = {
+    "tiny": dict(B=1, S=256, Hq=2, Hkv=2, d=64, D=2, seed=0, stress=0.0,
+                 desc="tiny: B=1 S=256 Hq=Hkv=2 d=64 D=2"),
+    "7b_mha": dict(B=1, S=16384, Hq=32, Hkv=32, d=128, D=8, seed=1, stress=0.0,
+                   desc="7B-dense MHA: B=1 S=16384 Hq=Hkv=32 d=128 D=8"),
+    "8b_gqa": dict(B=1, S=32768, Hq=32, Hkv=8, d=128, D=8, seed=2, stress=0.0,
+                   desc="Llama-3.1-8B-style GQA: B=1 S=32768 Hq=32 Hkv=8 d=128 D=8"),
+    "wide_gqa": dict(B=1, S=65536, Hq=24, Hkv=4, d=256, D=4, seed=3, stress=0.0,
+                     desc="wide-head GQA: B=1 S=65536 Hq=24 Hkv=4 d=256 D=4"),
+    "long": dict(B=1, S=131072, Hq=32, Hkv=8, d=128, D=16, seed=4, stress=0.001,
+                 desc="long context: B=1 S=131072 Hq=32 Hkv=8 d=128 D=16, 0.1% Q/K rows x8"),
+}
+DEFAULT_CONFIG = "7b_mha"
+# Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
+CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
+
+
+def fwd_flops(c, S=None):
+    S = c["S"] if S is None else S
+    return 4.0 * c["B"] * c["Hq"] * c["d"] * S * (S + 1) / 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk["bf16_tflops"], pk.get("bf16_tflops_sustained"), pk["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out = self.proc.communicate(timeout=10)[0]
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, smax, power, reasons = [], [], [], set()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(c, name):
+    """One bounded oracle step: full fwd + bwd at a reduced S. Returns (seconds, flops, desc)."""
+    import oracle
+    from sequence_sharded_causal_b200 import inputs
+    S = CPU_SAMPLE_S[name]
+    q_nat, k, v, do_nat, _ = inputs.make_inputs(c["B"], S, c["Hq"], c["Hkv"], c["d"], c["seed"])
+    perm, _ = oracle.partition(S, c["D"])
+    q = inputs.to_shard_major(q_nat, perm, c["D"])
+    do = inputs.to_shard_major(do_nat, perm, c["D"])
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, c["D"])
+    oracle.attn_bwd(q, k, v, do, c["D"])
+    dt = time.perf_counter() - t0
+    flops = 3.5 * fwd_flops(c, S)
+    desc = (f"oracle full fwd+bwd at S={S} (B={c['B']}, Hq={c['Hq']}, Hkv={c['Hkv']}, "
+            f"d={c['d']}, D={c['D']}), fp64")
+    return dt, flops, desc
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, c, name):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    oracle._load()
+    for _ in range(args.warmup):
+        oracle_sample(c, name)
+    total_t, total_f, desc = 0.0, 0.0, ""
+    for _ in range(args.steps):
+        dt, fl, desc = oracle_sample(c, name)
+        total_t += dt
+        total_f += fl
+    value = total_f / total_t / 1e12
+    cores = host_cores()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": c["desc"], "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_zsa(args, c, name):
+    import torch
+    import sequence_sharded_causal_b200 as zsa
+    from sequence_sharded_causal_b200 import inputs
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    B, S, Hq, Hkv, d, D = (c[k] for k in ("B", "S", "Hq", "Hkv", "d", "D"))
+    problem = zsa.make_problem(B, S, Hq, Hkv, d, D, causal=True)
+    perm = zsa.zsa_partition(problem, want_schedule=False)["perm"]
+    q_nat, k, v, do_nat, _ = inputs.make_inputs(B, S, Hq, Hkv, d, c["seed"] + 1000 * rank,
+                                                c["stress"], device=dev)
+    q = inputs.to_shard_major(q_nat, perm, D)
+    do = inputs.to_shard_major(do_nat, perm, D)
+    del q_nat, do_nat
+    o = torch.empty_like(q)
+    lse = torch.empty(D, B, Hq, S // D, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_f = torch.empty(zsa.zsa_workspace_bytes(problem, 0), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(zsa.zsa_workspace_bytes(problem, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        zsa.zsa_attn_fwd(problem, q, k, v, o, lse, ws_f, stream=stream)
+        zsa.zsa_attn_bwd(problem, q, k, v, o, lse, do, dq, dk, dv, ws_b, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = zsa.zsa_device_status(ws_f) or zsa.zsa_device_status(ws_b)
+    if status != zsa.ZSA_OK:
+        raise RuntimeError(f"device status after warm-up: {zsa.status_string(status)}")
+
+    # per-step kernel events (forward kernel, backward preprocess / main / dQ convert)
+    K = args.steps
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(4)] for _ in range(K)]
+    for row in kev:
+        for b_, e_ in row:
+            b_.record(stream)
+            e_.record(stream)
+    torch.cuda.synchronize(dev)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)   # let the sampler start before the timed region
+    e0.record(stream)
+    for i in range(K):
+        for which in range(4):
+            zsa.zsa_trace_events(which, kev[i][which][0], kev[i][which][1])
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier()
+    for which in range(4):
+        zsa.zsa_trace_events(which, None, None)
+    status = zsa.zsa_device_status(ws_f) or zsa.zsa_device_status(ws_b)
+    if status != zsa.ZSA_OK:
+        raise RuntimeError(f"device status after timing: {zsa.status_string(status)}")
+    ms = e0.elapsed_time(e1) / K
+    kms = [statistics.mean(kev[i][w][0].elapsed_time(kev[i][w][1]) for i in range(K))
+           for w in range(4)]
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the API with host buffers (copies inside the timed region)
+    pin = dict(pin_memory=True)
+    h_in = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in (q, k, v, do)]
+    for hsrc, dsrc in zip(h_in, (q, k, v, do)):
+        hsrc.copy_(dsrc)
+    h_out = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in (o, lse, dq, dk, dv)]
+    bi = sum(x.numel() * x.element_size() for x in h_in)
+    bo = sum(x.numel() * x.element_size() for x in h_out)
+    K2 = max(1, min(K, 10))
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(K2):
+        for dst, src in zip((q, k, v, do), h_in):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(h_out, (o, lse, dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = x0.elapsed_time(x1) / K2
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_sus, hbm, peak_src = load_peaks()
+    ff = fwd_flops(c)
+    bf = 2.5 * ff
+    value = world * (ff + bf) / (ms * 1e-3) / 1e12
+    fwd_tf = ff / (kms[0] * 1e-3) / 1e12
+    bwd_ms = kms[1] + kms[2] + kms[3]
+    bwd_tf = bf / (bwd_ms * 1e-3) / 1e12
+    main_tf = bf / (kms[2] * 1e-3) / 1e12
+    # dominant kernel by time: forward kernel or backward main kernel
+    if kms[2] >= kms[0]:
+        dom, dom_tf = "zsa_bwd_kernel", main_tf
+    else:
+        dom, dom_tf = "zsa_fwd_kernel", fwd_tf
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": c["desc"], "B": B, "S": S, "Hq": Hq, "Hkv": Hkv, "d": d, "D": D,
+                   "causal": True, "parallelism": "replicas" if world > 1 else "single",
+                   "l2": f"inputs larger than L2 ({(q.numel() + k.numel() + v.numel() + do.numel()) * 2 / 2**20:.0f} MiB vs 126 MiB), no flush"},
+        "pct_of_peak": 100.0 * value / world / peak,
+        "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+        "kernel_ms": {"fwd": kms[0], "bwd_pre": kms[1], "bwd_main": kms[2], "dq_convert": kms[3]},
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": dom_tf, "peak": peak,
+                     "unit": "TFLOP/s", "frac": dom_tf / peak, "peak_source": f"{peak_src} bf16 burst",
+                     "frac_of_sustained": (dom_tf / peak_sus) if peak_sus else None,
+                     "traffic": None},
+        "e2e": {"value": world * (ff + bf) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
+        "gpu_launches": 4 * K,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle._load()
+        dt, fl, desc = oracle_sample(c, name)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(),
+                                "kind": "oracle", "sample": desc, "seconds": dt}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="zsa", choices=("zsa", "reference"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    c = CONFIGS[args.config]
+    _, world, _ = dist_env()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, c, args.config)
+    else:
+        run_zsa(args, c, args.config)
+
+
+if __name__ == "__main__":
+    main()

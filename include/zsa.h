@@ -146,6 +146,15 @@ ZSA_API int zsa_set_wait_limit_ns(uint64_t limit_ns);
  * undefined.  Call with 0 to restore normal operation. */
 ZSA_API int zsa_debug_inject_stall(int enable);
 
+/* Tracing hook: while set, every later launch of kernel `which` records the CUDA
+ * events `begin_event` / `end_event` (cudaEvent_t handles owned by the caller) on the
+ * launch stream immediately before / after the kernel, so the caller can time that
+ * kernel alone with cudaEventElapsedTime.  which: ZSA_TRACE_FWD (forward kernel),
+ * ZSA_TRACE_BWD_PRE (Delta preprocess), ZSA_TRACE_BWD_MAIN (backward main kernel),
+ * ZSA_TRACE_BWD_DQ (dQ conversion).  Pass NULL events to stop tracing that kernel. */
+enum { ZSA_TRACE_FWD = 0, ZSA_TRACE_BWD_PRE = 1, ZSA_TRACE_BWD_MAIN = 2, ZSA_TRACE_BWD_DQ = 3 };
+ZSA_API int zsa_trace_events(int which, void* begin_event, void* end_event);
+
 /* Static string for a status code. */
 ZSA_API const char* zsa_status_string(int status);
 

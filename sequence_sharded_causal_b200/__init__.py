@@ -30,7 +30,8 @@ ZSA_ERR_TIMEOUT = -6
 
 EXPORTED = ("zsa_partition", "zsa_workspace_bytes", "zsa_attn_fwd", "zsa_attn_bwd",
             "zsa_device_status", "zsa_set_wait_limit_ns", "zsa_debug_inject_stall",
-            "zsa_status_string")
+            "zsa_trace_events", "zsa_status_string")
+ZSA_TRACE_FWD, ZSA_TRACE_BWD_PRE, ZSA_TRACE_BWD_MAIN, ZSA_TRACE_BWD_DQ = 0, 1, 2, 3
 
 
 class zsa_problem(ctypes.Structure):
@@ -75,6 +76,7 @@ def lib():
         L.zsa_device_status.argtypes = [vp, vp]
         L.zsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.zsa_debug_inject_stall.argtypes = [ctypes.c_int]
+        L.zsa_trace_events.argtypes = [ctypes.c_int, vp, vp]
         L.zsa_status_string.argtypes = [ctypes.c_int]
         L.zsa_status_string.restype = ctypes.c_char_p
         for name in EXPORTED[:-1]:
@@ -178,6 +180,18 @@ def zsa_set_wait_limit_ns(limit_ns):
 
 def zsa_debug_inject_stall(enable):
     _check(lib().zsa_debug_inject_stall(int(bool(enable))), "zsa_debug_inject_stall")
+
+
+def zsa_trace_events(which, begin_event=None, end_event=None):
+    """Record torch.cuda.Event (or raw cudaEvent_t) pairs around kernel `which`."""
+    def raw(e):
+        if e is None or isinstance(e, int):
+            return e
+        if not e.cuda_event:   # torch creates the event lazily on first record
+            e.record()
+        return e.cuda_event
+    _check(lib().zsa_trace_events(int(which), raw(begin_event), raw(end_event)),
+           "zsa_trace_events")
 
 
 def zsa_status_string(status):

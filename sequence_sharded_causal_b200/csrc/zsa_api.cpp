@@ -25,6 +25,8 @@ using zsa::Schedule;
 constexpr size_t kStatusBytes = 256;
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_inject_stall{0};
+std::atomic<void*> g_trace_begin[4];
+std::atomic<void*> g_trace_end[4];
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -124,7 +126,25 @@ size_t bwd_workspace(const zsa_problem* p) {
 
 }  // namespace
 
+namespace zsa {
+TraceEvents trace_events(int which) {
+  TraceEvents t{nullptr, nullptr};
+  if (which >= 0 && which < 4) {
+    t.begin = static_cast<cudaEvent_t>(g_trace_begin[which].load());
+    t.end = static_cast<cudaEvent_t>(g_trace_end[which].load());
+  }
+  return t;
+}
+}  // namespace zsa
+
 extern "C" {
+
+int zsa_trace_events(int which, void* begin_event, void* end_event) {
+  if (which < 0 || which >= 4) return ZSA_ERR_INVALID;
+  g_trace_begin[which].store(begin_event);
+  g_trace_end[which].store(end_event);
+  return ZSA_OK;
+}
 
 const char* zsa_status_string(int status) {
   switch (status) {

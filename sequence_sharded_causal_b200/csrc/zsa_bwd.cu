@@ -659,10 +659,13 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
     int64_t blocks = (warps_needed + 7) / 8;
     if (blocks > int64_t(sms) * 16) blocks = int64_t(sms) * 16;
     if (blocks < 1) blocks = 1;
+    const TraceEvents tr = trace_events(1);
+    if (tr.begin) cudaEventRecord(tr.begin, stream);
     zsa_bwd_pre_kernel<HD><<<int(blocks), 256, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.o), reinterpret_cast<const __nv_bfloat16*>(a.dout),
         a.delta, a.dq_acc, pairs, a.Hq, twoC);
     cudaError_t e = cudaGetLastError();
+    if (tr.end) cudaEventRecord(tr.end, stream);
     if (e != cudaSuccess) return int(e);
   }
   // K3
@@ -705,17 +708,23 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
     attr_set = true;
   }
   const int grid = p.n_units < sms ? p.n_units : sms;
+  const TraceEvents tr = trace_events(2);
+  if (tr.begin) cudaEventRecord(tr.begin, stream);
   zsa_bwd_kernel<HD><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, p);
   cudaError_t e = cudaGetLastError();
+  if (tr.end) cudaEventRecord(tr.end, stream);
   if (e != cudaSuccess) return int(e);
   // K4
   {
     const int64_t n8 = rows * a.Hq * HD / 8;
     int64_t blocks = (n8 + 255) / 256;
     if (blocks > int64_t(sms) * 16) blocks = int64_t(sms) * 16;
+    const TraceEvents tr4 = trace_events(3);
+    if (tr4.begin) cudaEventRecord(tr4.begin, stream);
     zsa_dq_convert_kernel<<<int(blocks), 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq),
                                                             n8, a.scale);
     e = cudaGetLastError();
+    if (tr4.end) cudaEventRecord(tr4.end, stream);
   }
   return int(e);
 }

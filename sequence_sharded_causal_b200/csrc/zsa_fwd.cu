@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       const int64_t j = int64_t(u.tile[s]) * 128 + row;             // row within the shard
       const int64_t pos = j < prm.C ? int64_t(u.r) * prm.C + j
                                     : int64_t(2 * prm.D - 1 - u.r) * prm.C + (j - prm.C);
-      float m_run = -INFINITY, l_run = 0.f;
+      float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
       for (int n = 0; n < u.kend[s]; ++n) {
         ok = warp_wait(&bars.s_full[s], s_ph, wctx);
         s_ph ^= 1;
@@ -369,24 +369,34 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             mt = fmaxf(mt, x);
           }
         const float m_new = fmaxf(m_run, mt);
-        if (m_new > m_run + 8.0f) {
-          if (n > 0) {
-            // O was accumulated against the old max: scale it (and l) down.
-            const float alpha = ex2_approx(m_run - m_new);
-            l_run *= alpha;
-#pragma unroll 1
-            for (int c = 0; c < HD / 32; ++c) {
-              uint32_t orow[32];
-              tmem_ld32(tO + c * 32, orow);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
-              tmem_st32(tO + c * 32, orow);
-            }
-          }
+        // The running max moves only when it grows by more than 2^8; O was accumulated
+        // against the old max, so it (and l) are scaled down by alpha.  The decision is
+        // per row, but the TMEM access is warp-collective (.sync.aligned), so the whole
+        // warp takes the rescale branch when any of its rows needs it (alpha = 1 for the
+        // others).
+        float alpha = 1.0f;
+        const bool grow = m_new > m_run + 8.0f;       // always true at n == 0
+        if (grow) {
+          if (n > 0) alpha = ex2_approx(m_run - m_new);
           m_run = m_new;
         }
-        float lsum = 0.f;
+        if (__any_sync(0xffffffffu, grow && n > 0)) {
+          l_run *= alpha;
+          r_run *= alpha;
+#pragma unroll 1
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t orow[32];
+            tmem_ld32(tO + c * 32, orow);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+            tmem_st32(tO + c * 32, orow);
+          }
+        }
+        // two row sums: of the fp32 P (for lse) and of the bf16-rounded P the PV MMA
+        // consumes (normalises O, keeping it a convex combination of V rows: exact
+        // when one key dominates a row)
+        float lsum = 0.f, rsum = 0.f;
 #pragma unroll
         for (int c = 0; c < BK / 32; ++c) {
           uint32_t pk[16];
@@ -396,10 +406,12 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             const float p1 = ex2_approx(__uint_as_float(sr[c][2 * e + 1]) - m_run);
             lsum += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
+            rsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
           }
           tmem_st16(tS + c * 16, pk);     // P (bf16 pairs) over the S columns already read
         }
         l_run += lsum;
+        r_run += rsum;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -411,7 +423,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       o_ph ^= 1;
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.0f / l_run;
+      const float inv_l = 1.0f / r_run;
       const int64_t grow = (int64_t(u.r) * prm.B + u.b) * twoC + j;    // shard-major row
       __nv_bfloat16* orow_g = prm.o + (grow * prm.Hq + u.head[s]) * HD;
 #pragma unroll 1
@@ -485,8 +497,12 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = a.n_units < sms ? a.n_units : sms;
   if (grid <= 0) return int(cudaSuccess);
+  const TraceEvents tr = trace_events(0);
+  if (tr.begin) cudaEventRecord(tr.begin, stream);
   zsa_fwd_kernel<HD><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, p);
-  return int(cudaGetLastError());
+  const cudaError_t e = cudaGetLastError();
+  if (tr.end) cudaEventRecord(tr.end, stream);
+  return int(e);
 }
 
 }  // namespace

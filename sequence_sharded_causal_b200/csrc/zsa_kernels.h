@@ -50,6 +50,12 @@ inline void fwd_tiling(int d, int32_t* bq, int32_t* bk, int32_t* slots) {
   *slots = d <= 128 ? 2 : 1;
 }
 
+// Caller-owned CUDA events recorded around one kernel's launches (null = not traced).
+struct TraceEvents {
+  cudaEvent_t begin, end;
+};
+TraceEvents trace_events(int which);  // which: 0 fwd, 1 bwd pre, 2 bwd main, 3 dQ convert
+
 // Returns a cudaError_t (cudaSuccess on success).
 int launch_fwd(const FwdArgs& a, cudaStream_t stream);
 int launch_bwd(const BwdArgs& a, cudaStream_t stream);

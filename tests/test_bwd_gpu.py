@@ -56,6 +56,21 @@ def test_bwd_matches_oracle(oracle, B, S, Hq, Hkv, d, D, causal, seed):
     assert max(errs.values()) <= REL_TOL, errs
 
 
+@pytest.mark.parametrize("B,S,Hq,Hkv,d,D,seed,frac", [
+    (1, 2048, 4, 2, 128, 4, 41, 0.01), (1, 1024, 2, 2, 64, 2, 42, 0.02)])
+def test_bwd_stress_rows(oracle, B, S, Hq, Hkv, d, D, seed, frac):
+    q_nat, k, v, do_nat, pos = inputs.make_inputs(B, S, Hq, Hkv, d, seed, stress_frac=frac)
+    assert pos.numel() > 0
+    perm, _ = oracle.partition(S, D)
+    q = inputs.to_shard_major(q_nat, perm, D)
+    do = inputs.to_shard_major(do_nat, perm, D)
+    ref = oracle.attn_bwd(q, k, v, do, D)
+    dq, dk, dv = gpu_fwd_bwd(q, k, v, do, D, True)
+    errs = {n: rel_fro(x, ref[n]) for n, x in (("dq", dq), ("dk", dk), ("dv", dv))}
+    assert all(np.isfinite(x).all() for x in (dq, dk, dv))
+    assert max(errs.values()) <= REL_TOL, errs
+
+
 def test_bwd_wait_timeout_reports_status(oracle):
     B, S, Hq, Hkv, d, D = 1, 1024, 4, 2, 128, 2
     q_nat, k, v, do_nat, _ = inputs.make_inputs(B, S, Hq, Hkv, d, 21)
