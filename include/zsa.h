@@ -130,6 +130,33 @@ ZSA_API int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* 
                  const void* o, const float* lse, const void* dout, void* dq, void* dk,
                  void* dv, void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* Size of the fixed device scratch behind zsa_attn_bwd_noalloc (64 MiB per device). */
+#define ZSA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* Backward without a workspace argument and without allocating anything.  The pages
+ * have no counterpart to this call: it exists for callers that cannot allocate device
+ * memory where they call the backward, such as code running while a stream is being
+ * captured into a CUDA graph under a no-allocation rule, plugins inside a host
+ * runtime that owns and pre-plans all device memory, or C callers without an
+ * allocator of their own.  Arguments and results are those of zsa_attn_bwd; the
+ * scratch (status word, Delta, fp32 dQ accumulator) is a fixed static device array of
+ * ZSA_NOALLOC_SCRATCH_BYTES that every GPU using this call keeps until the process
+ * exits.
+ *  - Problems needing more scratch than that (zsa_workspace_bytes(problem, 1) >
+ *    ZSA_NOALLOC_SCRATCH_BYTES) return ZSA_ERR_WORKSPACE before anything is enqueued.
+ *  - All calls on a device share the array: calls whose GPU work overlaps (other
+ *    streams or host threads) race and produce wrong results.  Each call re-zeroes
+ *    what must start at zero.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make it before any stream
+ *    capture begins.
+ *  - Device-side wait timeouts of this call are not reported (its status word lives in
+ *    the static array); waits stay bounded. */
+ZSA_API int zsa_attn_bwd_noalloc(const zsa_problem* problem, const void* q, const void* k,
+                                 const void* v, const void* o, const float* lse,
+                                 const void* dout, void* dq, void* dk, void* dv,
+                                 void* cuda_stream);
+
 /* Synchronises `cuda_stream`, reads and clears the status word at the start of
  * `workspace`: ZSA_OK, or ZSA_ERR_TIMEOUT if a device-side wait gave up. */
 ZSA_API int zsa_device_status(void* workspace, void* cuda_stream);
