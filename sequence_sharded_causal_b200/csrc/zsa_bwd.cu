@@ -99,9 +99,16 @@ __global__ void __launch_bounds__(256) zsa_dq_convert_kernel(const float* __rest
 // ------------------------------------------------------------------ K3: main backward
 template <int HD>
 struct BwdCfg {
-  static constexpr int BKV = 128;   // keys per CTA tile (TMEM lanes)
-  static constexpr int BQ = 64;     // query rows per slot
-  static constexpr int KB = HD / 64;
+  static constexpr int BKV = 128;                   // keys per CTA tile (TMEM lanes)
+  static constexpr int BQ = HD == 256 ? 32 : 64;    // query rows per slot
+  static constexpr int HC = HD == 256 ? 128 : HD;   // d columns one unit accumulates (dK, dV)
+  static constexpr int NCHUNK = HD / HC;            // units per key tile
+  static constexpr int KB = HD / 64;                // 64-wide d blocks of K, V, Q, dO
+  static constexpr int CB = HC / 64;                // 64-wide d blocks per chunk
+  static constexpr int HALF = BQ / 2;               // slot columns per compute group
+  // dS for the dQ MMA: MN-major [keys][BQ] (BQ = 64, one 128-byte swizzle row per key)
+  // or K-major [BQ][keys] (BQ = 32)
+  static constexpr bool DS_KMAJOR = BQ < 64;
   static constexpr int NQST = 2;    // Q/dO stages
   static constexpr int KV_BYTES = BKV * HD * 2;          // K (or V) tile
   static constexpr int QT_BYTES = BQ * HD * 2;           // Q (or dO) slot tile
@@ -119,12 +126,12 @@ struct BwdCfg {
   static constexpr int WARP_MMA = 13;
   static constexpr int NTHREADS = 14 * 32;
   static constexpr uint32_t TM_DV = 0;
-  static constexpr uint32_t TM_DK = HD;
-  static constexpr uint32_t TM_ST = 2 * HD;        // two buffers of 64 columns
-  static constexpr uint32_t TM_DPT = 2 * HD + 128;
-  static constexpr uint32_t TM_DQT = 2 * HD + 192;
+  static constexpr uint32_t TM_DK = HC;
+  static constexpr uint32_t TM_ST = 2 * HC;             // two buffers of BQ columns
+  static constexpr uint32_t TM_DPT = 2 * HC + 2 * BQ;
+  static constexpr uint32_t TM_DQT = 2 * HC + 3 * BQ;
   static constexpr uint32_t TM_COLS = 512;
-  static_assert(2 * HD + 256 <= 512, "TMEM budget");
+  static_assert(2 * HC + 4 * BQ <= 512, "TMEM budget");
   static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 };
 
@@ -136,7 +143,8 @@ struct BwdParams {
   __nv_bfloat16* dv;
   int64_t S, C;
   int32_t B, Hq, Hkv, G, D, causal;
-  int32_t n_units, n_qtiles;  // n_qtiles = 64-row tiles per shard
+  int32_t n_units, n_qtiles;  // n_qtiles = BQ-row tiles per shard
+  int32_t n_chunks, bq;       // d chunks per key tile, query rows per slot
   float scale, scale_log2;
   int* status;
   uint64_t wait_limit_ns;
@@ -157,7 +165,7 @@ struct BwdBars {
 
 // One key tile of work.
 struct KvUnit {
-  int32_t n, b, g;
+  int32_t n, b, g, c;   // key tile, batch, kv head, d chunk
 };
 
 __device__ __forceinline__ int bwd_unit_index(int k, int n_units) {
@@ -166,20 +174,23 @@ __device__ __forceinline__ int bwd_unit_index(int k, int n_units) {
   return idx < n_units ? idx : -1;
 }
 
-__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int B, int Hkv) {
+// Units in order of key tile n (most work first), then b, g, d chunk.
+__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int B, int Hkv, int NC) {
   KvUnit u;
-  u.n = idx / (B * Hkv);
-  const int rem = idx % (B * Hkv);
-  u.b = rem / Hkv;
-  u.g = rem % Hkv;
+  u.n = idx / (B * Hkv * NC);
+  const int rem = idx % (B * Hkv * NC);
+  u.b = rem / (Hkv * NC);
+  u.g = (rem / NC) % Hkv;
+  u.c = rem % NC;
   return u;
 }
 
-// Enumerates the q slots (shard r, 64-row tile i, head offset e) that see key tile n,
-// in (r, i, e) order.  Every role walks the same sequence.
+// Enumerates the q slots (shard r, BQ-row tile i, head offset e) that see key tile n,
+// in (r, i, e) order.  Every role walks the same sequence.  A BQ-row tile never
+// straddles a zigzag chunk (C is a multiple of 64), so its positions are contiguous.
 struct SlotWalk {
   int32_t r, i, e;
-  int64_t p0;   // position of the tile's first row (its rows are p0 .. p0+63)
+  int64_t p0;   // position of the tile's first row (its rows are p0 .. p0+BQ-1)
 };
 
 __device__ __forceinline__ int64_t zz_pos(int64_t C, int32_t D, int32_t r, int64_t j) {
@@ -188,8 +199,8 @@ __device__ __forceinline__ int64_t zz_pos(int64_t C, int32_t D, int32_t r, int64
 
 __device__ __forceinline__ bool tile_sees(const BwdParams& p, int32_t r, int32_t i, int32_t n,
                                           int64_t* p0) {
-  *p0 = zz_pos(p.C, p.D, r, int64_t(i) * 64);
-  return !p.causal || (*p0 + 63 >= int64_t(n) * 128);
+  *p0 = zz_pos(p.C, p.D, r, int64_t(i) * p.bq);
+  return !p.causal || (*p0 + p.bq - 1 >= int64_t(n) * 128);
 }
 
 // First slot at or after (r, i, 0); false when the walk is over.
@@ -229,7 +240,8 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
                    const __grid_constant__ CUtensorMap map_v,
                    const __grid_constant__ CUtensorMap map_do, const BwdParams prm) {
   using Cfg = BwdCfg<HD>;
-  constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV;
+  constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV, HC = Cfg::HC, CB = Cfg::CB;
+  constexpr int HALF = Cfg::HALF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -287,7 +299,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
       for (int k = 0; ok; ++k) {
         const int idx = bwd_unit_index(k, prm.n_units);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
         if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
@@ -331,8 +343,8 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16(128, BQ, false, false);
-      const uint32_t idesc_kv = idesc_bf16(128, HD, false, true);
-      const uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);
+      const uint32_t idesc_kv = idesc_bf16(128, HC, false, true);
+      const uint32_t idesc_dq = idesc_bf16(128, BQ, true, !Cfg::DS_KMAJOR);
       const uint32_t sK = smem_u32(smem + Cfg::SMEM_K);
       const uint32_t sV = smem_u32(smem + Cfg::SMEM_V);
       const uint32_t sQ = smem_u32(smem + Cfg::SMEM_Q);
@@ -350,6 +362,11 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
       uint32_t acc_commits = 0;
       bool ok = true;
       if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
+      // TMEM column (bf16 pairs) of q columns 16ks .. 16ks+15 of P^T / dS^T: compute
+      // group h writes its HALF columns as HALF/2 packed columns at h*HALF
+      auto p_col = [](int ks) -> uint32_t {
+        return uint32_t(((16 * ks) / HALF) * HALF + ((16 * ks) % HALF) / 2);
+      };
       auto wait_st_free = [&](int b) {
         if (st_commits[b] > st_waits[b]) {
           ok = ok && mbar_wait(&bars.st_free[b], st_waits[b] & 1, wctx);
@@ -366,7 +383,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
         for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + Cfg::TM_ST + b * 64, sdesc_sw128(sK + kb * BKV * 128 + ks * 32, 16, 1024),
+            mma_ss(tmem + Cfg::TM_ST + b * BQ, sdesc_sw128(sK + kb * BKV * 128 + ks * 32, 16, 1024),
                    sdesc_sw128(sQ + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
                    idesc_s, (kb | ks) != 0);
       };
@@ -381,7 +398,9 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
       for (int k = 0; ok; ++k) {
         const int idx = bwd_unit_index(k, prm.n_units);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
+        const uint32_t cq = uint32_t(u.c * CB * BQ * 128);   // chunk offset in a Q / dO tile
+        const uint32_t ck = uint32_t(u.c * CB * BKV * 128);  // chunk offset in the K tile
         ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
         kv_ph ^= 1;
         if (!ok) break;
@@ -418,8 +437,8 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < BQ / 16; ++ks)
-            mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + b * 64 + (ks >> 1) * 32 + (ks & 1) * 8,
-                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+            mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + b * BQ + p_col(ks),
+                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + cq + ks * 2048, BQ * 128, 1024), idesc_kv,
                    (j > 0) || (ks > 0));
           mma_commit(&bars.st_free[b]);
           ++st_commits[b];
@@ -440,8 +459,8 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < BQ / 16; ++ks)
-            mma_ts(tmem + Cfg::TM_DK, tmem + Cfg::TM_DPT + (ks >> 1) * 32 + (ks & 1) * 8,
-                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+            mma_ts(tmem + Cfg::TM_DK, tmem + Cfg::TM_DPT + p_col(ks),
+                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + cq + ks * 2048, BQ * 128, 1024), idesc_kv,
                    (j > 0) || (ks > 0));
           mma_commit(&bars.dpt_free);
           ++dpt_commits;
@@ -452,10 +471,14 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
             tc_fence_after();
           }
 #pragma unroll
-          for (int ks = 0; ks < BKV / 16; ++ks)
-            mma_ss(tmem + Cfg::TM_DQT, sdesc_sw128(sK + ks * 2048, lbo_kt, 1024),
-                   sdesc_sw128(sDS + b * Cfg::DS_BYTES + ks * 2048, BQ * 128, 1024), idesc_dq,
-                   ks > 0);
+          for (int ks = 0; ks < BKV / 16; ++ks) {
+            const uint64_t bdesc =
+                Cfg::DS_KMAJOR
+                    ? sdesc_sw128(sDS + b * Cfg::DS_BYTES + (ks >> 2) * BQ * 128 + (ks & 3) * 32, 16, 1024)
+                    : sdesc_sw128(sDS + b * Cfg::DS_BYTES + ks * 2048, BQ * 128, 1024);
+            mma_ss(tmem + Cfg::TM_DQT, sdesc_sw128(sK + ck + ks * 2048, lbo_kt, 1024), bdesc,
+                   idesc_dq, ks > 0);
+          }
           mma_commit(&bars.dq_full);
           ++dq_commits;
           mma_commit(&bars.dsm_free[b]);
@@ -484,42 +507,43 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
   } else if (warp >= Cfg::WARP_DQ) {
     // ------------------------------------------------------------ dQ warps
     const int qw = warp - Cfg::WARP_DQ;
-    const int drow = qw * 32 + lane;           // TMEM lane = d index of dQ^T
+    const int drow = qw * 32 + lane;           // TMEM lane = d index (within the chunk) of dQ^T
     const uint32_t tDQ = tmem + Cfg::TM_DQT + (uint32_t(qw * 32) << 16);
     uint32_t dq_ph = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int idx = bwd_unit_index(k, prm.n_units);
       if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
       SlotWalk w;
       for (bool more = walk_first(prm, u.n, w); more; more = walk_next(prm, u.n, w)) {
         ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
         dq_ph ^= 1;
         if (!ok) break;
         tc_fence_after();
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tDQ, v0);
-        tmem_ld32(tDQ + 32, v1);
+        uint32_t v[BQ / 32][32];
+#pragma unroll
+        for (int t = 0; t < BQ / 32; ++t) tmem_ld32(tDQ + t * 32, v[t]);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.dq_empty);
-        if (drow < HD) {
+        if (drow < HC) {
           const int32_t h = u.g * prm.G + w.e;
           const int64_t row0 = (int64_t(w.r) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
-          float* base = prm.dq_acc + (row0 * prm.Hq + h) * HD + drow;
+          float* base = prm.dq_acc + (row0 * prm.Hq + h) * HD + u.c * HC + drow;
           const int64_t rstride = int64_t(prm.Hq) * HD;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) atomicAdd(base + c * rstride, __uint_as_float(v0[c]));
+          for (int t = 0; t < BQ / 32; ++t)
 #pragma unroll
-          for (int c = 0; c < 32; ++c) atomicAdd(base + (32 + c) * rstride, __uint_as_float(v1[c]));
+            for (int c = 0; c < 32; ++c)
+              atomicAdd(base + (t * 32 + c) * rstride, __uint_as_float(v[t][c]));
         }
       }
     }
   } else {
     // ------------------------------------------------------------ compute warps
-    const int half = warp / 4;                 // which 32 of the slot's 64 columns
+    const int half = warp / 4;                 // which HALF of the slot's BQ columns
     const int qw = warp % 4;
     const int row = qw * 32 + lane;            // TMEM lane = key within the tile
     const uint32_t lane_addr = uint32_t(qw * 32) << 16;
@@ -533,7 +557,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
     for (int k = 0; ok; ++k) {
       const int idx = bwd_unit_index(k, prm.n_units);
       if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv);
+      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
       const int64_t key = int64_t(u.n) * BKV + row;
       SlotWalk w;
       int j = 0;
@@ -544,29 +568,29 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
         ++q_full_uses[st];
         if (!ok) break;
         // per-column statistics of this warp's 32 query rows, read from shared memory
-        const float* lse_c = sLse + st * BQ + half * 32;
-        const float* dlt_c = sDelta + st * BQ + half * 32;
-        // causal mask: column c holds position p0 + half*32 + c; masked when key > it
-        const int64_t first = w.p0 + half * 32;
+        const float* lse_c = sLse + st * BQ + half * HALF;
+        const float* dlt_c = sDelta + st * BQ + half * HALF;
+        // causal mask: column c holds position p0 + half*HALF + c; masked when key > it
+        const int64_t first = w.p0 + half * HALF;
         const int nvis_lo = prm.causal ? int(key - first) : 0;   // columns c < nvis_lo are masked
         // ---- P^T
         ok = warp_wait_b(&bars.s_full[b], s_ph[b], wctx);
         s_ph[b] ^= 1;
         if (!ok) break;
         tc_fence_after();
-        uint32_t sv[32];
-        tmem_ld32(tmem + Cfg::TM_ST + b * 64 + half * 32 + lane_addr, sv);
+        uint32_t sv[HALF];
+        tmem_ld_n<HALF>(tmem + Cfg::TM_ST + b * BQ + half * HALF + lane_addr, sv);
         tmem_ld_wait();
-        float pf[32];
-        uint32_t pk[16];
+        float pf[HALF];
+        uint32_t pk[HALF / 2];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < HALF; ++c) {
           const float x = fmaf(__uint_as_float(sv[c]), prm.scale_log2, -lse_c[c] * kLog2e);
           pf[c] = (c < nvis_lo) ? 0.f : ex2_approx(x);
         }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
-        tmem_st16(tmem + Cfg::TM_ST + b * 64 + half * 32 + lane_addr, pk);
+        for (int e = 0; e < HALF / 2; ++e) pk[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
+        tmem_st_n<HALF / 2>(tmem + Cfg::TM_ST + b * BQ + half * HALF + lane_addr, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -576,27 +600,43 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
         dp_ph ^= 1;
         if (!ok) break;
         tc_fence_after();
-        tmem_ld32(tmem + Cfg::TM_DPT + half * 32 + lane_addr, sv);
+        tmem_ld_n<HALF>(tmem + Cfg::TM_DPT + half * HALF + lane_addr, sv);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
+        for (int e = 0; e < HALF / 2; ++e)
           pk[e] = pack_bf16x2(pf[2 * e] * (__uint_as_float(sv[2 * e]) - dlt_c[2 * e]),
                               pf[2 * e + 1] * (__uint_as_float(sv[2 * e + 1]) - dlt_c[2 * e + 1]));
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.q_empty[st]);   // lse / Delta of this stage consumed
         ++q_it;
-        tmem_st16(tmem + Cfg::TM_DPT + half * 32 + lane_addr, pk);
-        // shared-memory copy for dQ^T: row = key, 16-byte chunks 4*half .. 4*half+3
+        tmem_st_n<HALF / 2>(tmem + Cfg::TM_DPT + half * HALF + lane_addr, pk);
+        // shared-memory copy of dS for the dQ MMA
         if (dsm_uses[b] > 0) {
           ok = warp_wait_b(&bars.dsm_free[b], (dsm_uses[b] - 1) & 1, wctx);
           if (!ok) break;
         }
         ++dsm_uses[b];
         uint8_t* dsb = sDS + b * Cfg::DS_BYTES;
+        if constexpr (!Cfg::DS_KMAJOR) {
+          // MN-major [key][64 q]: row = key, 16-byte chunks 4*half .. 4*half+3
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<uint4*>(dsb + sw128_offset(uint32_t(row), uint32_t(4 * half + m))) =
-              make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+          for (int m = 0; m < 4; ++m)
+            *reinterpret_cast<uint4*>(dsb + sw128_offset(uint32_t(row), uint32_t(4 * half + m))) =
+                make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+        } else {
+          // K-major [q][keys] in 64-key blocks of BQ rows x 128 B: element (q, key) sits
+          // in block key/64, row q, 16-byte chunk ((key%64)/8) ^ (q%8), bytes 2*(key%8)
+          uint8_t* blk = dsb + (row >> 6) * (BQ * 128);
+          const uint32_t kc = uint32_t((row & 63) >> 3), kb2 = uint32_t((row & 7) * 2);
+#pragma unroll
+          for (int e = 0; e < HALF / 2; ++e) {
+            const uint32_t q0 = uint32_t(half * HALF + 2 * e);
+            *reinterpret_cast<uint16_t*>(blk + q0 * 128 + ((kc ^ (q0 & 7)) << 4) + kb2) =
+                uint16_t(pk[e] & 0xFFFFu);
+            *reinterpret_cast<uint16_t*>(blk + (q0 + 1) * 128 + ((kc ^ ((q0 + 1) & 7)) << 4) + kb2) =
+                uint16_t(pk[e] >> 16);
+          }
+        }
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
@@ -612,9 +652,9 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
       const uint32_t tAcc = tmem + (half == 0 ? Cfg::TM_DV : Cfg::TM_DK) + lane_addr;
       const float mul = half == 0 ? 1.0f : prm.scale;
       __nv_bfloat16* dst = (half == 0 ? prm.dv : prm.dk) +
-                           ((int64_t(u.b) * prm.S + key) * prm.Hkv + u.g) * HD;
+                           ((int64_t(u.b) * prm.S + key) * prm.Hkv + u.g) * HD + u.c * HC;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = 0; c < HC / 32; ++c) {
         uint32_t a[32];
         tmem_ld32(tAcc + c * 32, a);
         tmem_ld_wait();
@@ -693,8 +733,10 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.S = a.S;
   p.C = a.S / (2 * int64_t(a.D));
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = a.Hq / a.Hkv; p.D = a.D; p.causal = a.causal;
-  p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / Cfg::BKV));
+  p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / Cfg::BKV) * Cfg::NCHUNK);
   p.n_qtiles = int32_t(twoC / Cfg::BQ);
+  p.n_chunks = Cfg::NCHUNK;
+  p.bq = Cfg::BQ;
   p.scale = a.scale;
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
   p.status = a.status;
@@ -735,6 +777,7 @@ int launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   switch (a.d) {
     case 64: return launch_bwd_hd<64>(a, stream);
     case 128: return launch_bwd_hd<128>(a, stream);
+    case 256: return launch_bwd_hd<256>(a, stream);
     default: return int(cudaErrorNotSupported);
   }
 }

@@ -25,6 +25,9 @@ CASES = [  # (B, S, Hq, Hkv, d, D, causal, seed)
     (1, 1536, 4, 1, 128, 3, True, 6),      # GQA 4, D = 3
     (1, 1024, 4, 4, 128, 1, True, 7),      # D = 1
     (1, 2048, 4, 2, 64, 8, True, 8),       # D = 8
+    (1, 1024, 6, 1, 256, 2, True, 9),      # d = 256 (two d-chunk units per key tile), GQA 6
+    (1, 512, 4, 2, 256, 2, True, 10),      # d = 256, 32-row q slots, C = 128
+    (2, 512, 2, 2, 256, 1, False, 11),     # d = 256, non-causal, D = 1, B = 2
 ]
 
 
@@ -57,7 +60,8 @@ def test_bwd_matches_oracle(oracle, B, S, Hq, Hkv, d, D, causal, seed):
 
 
 @pytest.mark.parametrize("B,S,Hq,Hkv,d,D,seed,frac", [
-    (1, 2048, 4, 2, 128, 4, 41, 0.01), (1, 1024, 2, 2, 64, 2, 42, 0.02)])
+    (1, 2048, 4, 2, 128, 4, 41, 0.01), (1, 1024, 2, 2, 64, 2, 42, 0.02),
+    (1, 1024, 6, 1, 256, 2, 43, 0.02)])
 def test_bwd_stress_rows(oracle, B, S, Hq, Hkv, d, D, seed, frac):
     q_nat, k, v, do_nat, pos = inputs.make_inputs(B, S, Hq, Hkv, d, seed, stress_frac=frac)
     assert pos.numel() > 0
