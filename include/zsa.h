@@ -105,8 +105,8 @@ typedef struct {
  * Tiling: q tile i of shard r covers rows [i*block_q, (i+1)*block_q) of the shard;
  * its k_tile_end is (largest position in the tile)/block_k + 1 (causal) or S/block_k.
  * Units list, per (b, kv head g, shard r), the tile-major slots s = i*G + e (q head
- * g*G + e) in consecutive runs of `slots`; they are ordered by max k_tile_end
- * descending, then shard, then run index, then b, then g (all ascending).
+ * g*G + e) in consecutive runs of `slots`; they are ordered by b, then g (ascending),
+ * and within one (b, g) by max k_tile_end descending, then shard, then run index.
  * Returns ZSA_ERR_WORKSPACE when cap < *n_work_out and sched_host != NULL.
  */
 ZSA_API int zsa_partition(const zsa_problem* problem, zsa_tiling* tiling, int32_t* perm_host,

@@ -88,8 +88,8 @@ int oracle_partition(int64_t S, int32_t D, int32_t *perm, int32_t *inv_perm)
  * runs of `slots` slots form one unit (the last run may be short).  A unit row is
  *   {r, b, g, tile0, head0, tile1, head1, kend0, kend1}
  * with -1 / 0 for absent slots (slots == 1 leaves the second slot absent).
- * Order: by max(kend0, kend1) descending, then r, then the unit's index m within
- * its (b, g, r) list, then b, then g, all ascending.
+ * Order: by b, then g (ascending); within one (b, g) by max(kend0, kend1)
+ * descending, then r, then the unit's index m within its (b, g, r) list (ascending).
  */
 typedef struct {
     int32_t f[9];
@@ -99,11 +99,11 @@ typedef struct {
 static int unit_cmp(const void *pa, const void *pb)
 {
     const unit_rec *a = (const unit_rec *)pa, *b = (const unit_rec *)pb;
+    if (a->key_b != b->key_b) return a->key_b < b->key_b ? -1 : 1;
+    if (a->key_g != b->key_g) return a->key_g < b->key_g ? -1 : 1;
     if (a->key_work != b->key_work) return a->key_work > b->key_work ? -1 : 1;
     if (a->key_r != b->key_r) return a->key_r < b->key_r ? -1 : 1;
     if (a->key_m != b->key_m) return a->key_m < b->key_m ? -1 : 1;
-    if (a->key_b != b->key_b) return a->key_b < b->key_b ? -1 : 1;
-    if (a->key_g != b->key_g) return a->key_g < b->key_g ? -1 : 1;
     return 0;
 }
 

@@ -6,8 +6,9 @@
 // sharing kv heads ("Tensor, pipeline e sequence parallelism", 01 Conceito).  The
 // pages give no kernel design; this one is built for the B200:
 //
-//  * persistent CTAs, one per SM, walk the host-built unit table (units sorted by
-//    work, longest first, assigned in snake order);
+//  * persistent CTAs, one per SM, claim units of the host-built table from a global
+//    counter (the table is grouped by (b, kv head), longest first within a group, so
+//    CTAs busy at the same time share one head's K/V in L2);
 //  * a unit is up to NSLOT (q tile, q head) slots of 128 query rows that share one K/V
 //    stream: two q heads of one kv group (GQA) or two adjacent q tiles (MHA), so a
 //    K/V tile fetched once feeds 2 x 128 rows of MMAs;
@@ -66,14 +67,18 @@ struct FwdParams {
   int32_t B, Hq, Hkv, D, causal;
   float scale_log2;
   int* status;
+  int* counter;       // next unclaimed unit (zeroed before every launch)
   uint64_t wait_limit_ns;
   int inject_stall;
 };
+
+constexpr int kUnitRing = 4;  // claimed units in flight between the producer and the others
 
 struct FwdBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t drain;
   uint64_t never;  // test hook: no one ever arrives here
 };
@@ -96,12 +101,6 @@ __device__ __forceinline__ UnitInfo load_unit(const DevUnit* units, int idx) {
   return u;
 }
 
-// k-th unit of this CTA in snake order over stripes of gridDim.x units; -1 when done.
-__device__ __forceinline__ int unit_index(int k, int n_units) {
-  const int grid = int(gridDim.x);
-  const int idx = k * grid + ((k & 1) ? (grid - 1 - int(blockIdx.x)) : int(blockIdx.x));
-  return idx < n_units ? idx : -1;
-}
 
 // Every lane polls; the outcome is made warp-uniform so .sync.aligned TMEM ops that
 // follow are executed by the full warp or by none of it.
@@ -123,6 +122,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
   __shared__ FwdBars bars;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ int unit_ring[kUnitRing];
 
   const int warp = int(warp_id()), lane = int(lane_id());
   if (threadIdx.x == 0) {
@@ -141,6 +141,10 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       mbar_init(&bars.k_empty[s], 1);
       mbar_init(&bars.v_full[s], 1);
       mbar_init(&bars.v_empty[s], 1);
+    }
+    for (int s = 0; s < kUnitRing; ++s) {
+      mbar_init(&bars.unit_full[s], 1);
+      mbar_init(&bars.unit_empty[s], 1 + 4 * Cfg::NSLOT);   // MMA thread + softmax warps
     }
     mbar_init(&bars.drain, 1);
     mbar_init(&bars.never, 1);
@@ -174,7 +178,16 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       for (int st = 0; st < ST; ++st) k_fills[st] = v_fills[st] = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int idx = unit_index(k, prm.n_units);
+        // Claim the next unit of the table (dynamic scheduling: the table is grouped
+        // by kv head, so CTAs busy at the same time share that head's K/V in L2) and
+        // hand it to the MMA thread and the softmax warps through the ring.
+        const int slot = k % kUnitRing;
+        if (k >= kUnitRing) ok = mbar_wait(&bars.unit_empty[slot], ((k / kUnitRing) - 1) & 1, wctx);
+        if (!ok) break;
+        int idx = atomicAdd(prm.counter, 1);
+        if (idx >= prm.n_units) idx = -1;
+        unit_ring[slot] = idx;
+        mbar_arrive(&bars.unit_full[slot]);
         if (idx < 0) break;
         const UnitInfo u = load_unit(prm.units, idx);
         for (int s = 0; s < NSLOT && ok; ++s) {
@@ -248,7 +261,11 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         }
       };
       for (int k = 0; ok; ++k) {
-        const int idx = unit_index(k, prm.n_units);
+        const int slot = k % kUnitRing;
+        ok = mbar_wait(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+        if (!ok) break;
+        const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+        mbar_arrive(&bars.unit_empty[slot]);
         if (idx < 0) break;
         const UnitInfo u = load_unit(prm.units, idx);
         for (int s = 0; s < NSLOT && ok; ++s) {
@@ -339,7 +356,12 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
     uint32_t s_ph = 0, o_ph = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = unit_index(k, prm.n_units);
+      const int slot = k % kUnitRing;
+      ok = warp_wait(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+      if (!ok) break;
+      const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
       if (idx < 0) break;
       const UnitInfo u = load_unit(prm.units, idx);
       if (u.kend[s] == 0) continue;
@@ -356,24 +378,32 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
 #pragma unroll
         for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
         tmem_ld_wait();
-        const int64_t key0 = int64_t(n) * BK;
-        const bool masked = prm.causal && (key0 + BK - 1 > pos);
-        float mt = -INFINITY;
+        // Causal mask on the tiles that cross this warp's diagonal only: keys past
+        // `lim` (relative to the tile) are invisible to this row.  Off-diagonal tiles
+        // (all but about one in kend) skip the mask entirely.
+        const int64_t rel = pos - int64_t(n) * BK;
+        const int lim = rel >= BK ? BK : int(rel);              // >= 0: key 0 is always visible
+        if (prm.causal && __any_sync(0xffffffffu, lim < BK - 1)) {
+#pragma unroll
+          for (int c = 0; c < BK / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e > lim) sr[c][e] = 0xFF800000u;    // -inf
+        }
+        // row max of the raw scores (three-input max, four independent chains)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < BK / 32; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float x = __uint_as_float(sr[c][e]) * prm.scale_log2;
-            if (masked && key0 + c * 32 + e > pos) x = -INFINITY;
-            sr[c][e] = __float_as_uint(x);
-            mt = fmaxf(mt, x);
-          }
-        const float m_new = fmaxf(m_run, mt);
-        // The running max moves only when it grows by more than 2^8; O was accumulated
-        // against the old max, so it (and l) are scaled down by alpha.  The decision is
-        // per row, but the TMEM access is warp-collective (.sync.aligned), so the whole
-        // warp takes the rescale branch when any of its rows needs it (alpha = 1 for the
-        // others).
+          for (int e = 0; e < 32; e += 2)
+            mx[(e >> 1) & 3] = max3f(mx[(e >> 1) & 3], __uint_as_float(sr[c][e]),
+                                     __uint_as_float(sr[c][e + 1]));
+        const float m_new = fmaxf(m_run, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * prm.scale_log2);
+        // The running max (log2 units) moves only when it grows by more than 2^8; O was
+        // accumulated against the old max, so it (and l) are scaled down by alpha.  The
+        // decision is per row, but the TMEM access is warp-collective (.sync.aligned),
+        // so the whole warp takes the rescale branch when any of its rows needs it
+        // (alpha = 1 for the others).
         float alpha = 1.0f;
         const bool grow = m_new > m_run + 8.0f;       // always true at n == 0
         if (grow) {
@@ -393,25 +423,36 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             tmem_st32(tO + c * 32, orow);
           }
         }
-        // two row sums: of the fp32 P (for lse) and of the bf16-rounded P the PV MMA
-        // consumes (normalises O, keeping it a convex combination of V rows: exact
-        // when one key dominates a row)
-        float lsum = 0.f, rsum = 0.f;
+        // P = 2^(s*scale*log2e - m), two elements per packed FMA.  Two row sums, in
+        // packed adds: of the fp32 P (for lse) and of the bf16-rounded P the PV MMA
+        // consumes (normalises O, keeping it a convex combination of V rows: exact when
+        // one key dominates a row).
+        const uint64_t scale2 = f2_pack(prm.scale_log2, prm.scale_log2);
+        const uint64_t negm2 = f2_pack(-m_run, -m_run);
+        uint64_t lsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        uint64_t rsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < BK / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(__uint_as_float(sr[c][2 * e]) - m_run);
-            const float p1 = ex2_approx(__uint_as_float(sr[c][2 * e + 1]) - m_run);
-            lsum += p0 + p1;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
+                                       scale2, negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            lsum2[e & 1] = f2_add(lsum2[e & 1], f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
-            rsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+            rsum2[e & 1] = f2_add(rsum2[e & 1], bf16x2_widen(pk[e]));
           }
           tmem_st16(tS + c * 16, pk);     // P (bf16 pairs) over the S columns already read
         }
-        l_run += lsum;
-        r_run += rsum;
+        float a0, a1, b0, b1;
+        f2_unpack(f2_add(lsum2[0], lsum2[1]), a0, a1);
+        f2_unpack(f2_add(rsum2[0], rsum2[1]), b0, b1);
+        l_run += a0 + a1;
+        r_run += b0 + b1;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -483,6 +524,7 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.D = a.D; p.causal = a.causal;
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
   p.status = a.status;
+  p.counter = a.status + 32;
   p.wait_limit_ns = a.wait_limit_ns;
   p.inject_stall = a.inject_stall;
   const int smem = Cfg::SMEM_BYTES + 1024;

@@ -69,12 +69,14 @@ bool build_schedule(int64_t S, int32_t D, int32_t B, int32_t Hq, int32_t Hkv, in
           x.r = r; x.m = int32_t(m); x.b = b; x.g = g;
           list.push_back(x);
         }
+  // Grouped by (b, kv head) so that units running at the same time share one head's
+  // K/V in L2; longest first within a group so each group ends with its shortest units.
   std::sort(list.begin(), list.end(), [](const Keyed& a, const Keyed& c) {
+    if (a.b != c.b) return a.b < c.b;
+    if (a.g != c.g) return a.g < c.g;
     if (a.work != c.work) return a.work > c.work;
     if (a.r != c.r) return a.r < c.r;
-    if (a.m != c.m) return a.m < c.m;
-    if (a.b != c.b) return a.b < c.b;
-    return a.g < c.g;
+    return a.m < c.m;
   });
   out->units.resize(list.size());
   for (size_t k = 0; k < list.size(); ++k) out->units[k] = list[k].u;

@@ -77,7 +77,8 @@ def _pins_pass():
         if k0 != int(rows.max()) // bk + 1:
             return False
     work = np.maximum(units[:, 7], units[:, 8])
-    if not (np.diff(work) <= 0).all():
+    grp = units[:, 1] * 1 + units[:, 2]
+    if not (np.diff(grp) >= 0).all() or not (np.diff(work)[np.diff(grp) == 0] <= 0).all():
         return False
     # forward vs unsharded brute force (GQA, causal)
     B, S, Hq, Hkv, d, D = 1, 32, 4, 2, 8, 2

@@ -133,7 +133,10 @@ def test_schedule_brute(oracle, S, D, B, Hq, Hkv, bq, bk):
                     seen.add((r, b, i1, h1))
             assert len(seen) == D * B * T * Hq
             work = np.maximum(units[:, 7], units[:, 8])
-            assert (np.diff(work) <= 0).all()
+            grp = units[:, 1] * Hkv + units[:, 2]
+            assert (np.diff(grp) >= 0).all()                      # (b, g)-major
+            same = np.diff(grp) == 0
+            assert (np.diff(work)[same] <= 0).all()               # longest first within a group
 
 
 @pytest.mark.parametrize("S,D,Hq,Hkv,bq,bk,per_head", [
