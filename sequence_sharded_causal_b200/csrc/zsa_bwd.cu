@@ -14,8 +14,9 @@
 // summed across key tiles with fp32 reductions into a workspace accumulator.
 //
 // K3 layout (d = 128; d = 64 uses the same code with half-width accumulators):
-//  * one persistent CTA per SM walks key tiles (n ascending = most work first; snake
-//    order over CTAs); K and V (128 keys) stay in shared memory for the whole tile;
+//  * one persistent CTA per SM claims key-tile units from a global counter, grouped by
+//    (b, kv head) and longest first within a group; K and V (128 keys) stay in shared
+//    memory for the whole tile;
 //  * q slots are 64-row tiles (a 64-row tile never straddles a zigzag chunk because
 //    C is a multiple of 64) streamed through a 2-stage ring: Q, dO, lse, Delta;
 //  * TMEM: dV | dK (fp32, 128 lanes = keys) | S^T x2 | dP^T | dQ^T (64 cols each);
@@ -145,11 +146,15 @@ struct BwdParams {
   int32_t B, Hq, Hkv, G, D, causal;
   int32_t n_units, n_qtiles;  // n_qtiles = BQ-row tiles per shard
   int32_t n_chunks, bq;       // d chunks per key tile, query rows per slot
+  int32_t n_ktiles;           // S / 128
   float scale, scale_log2;
   int* status;
+  int* counter;       // next unclaimed unit (zeroed before every launch)
   uint64_t wait_limit_ns;
   int inject_stall;
 };
+
+constexpr int kUnitRing = 4;   // claimed units in flight between the producer and the others
 
 struct BwdBars {
   uint64_t kv_full, kv_empty;
@@ -160,6 +165,7 @@ struct BwdBars {
   uint64_t dsm_free[2];
   uint64_t dq_full, dq_empty;
   uint64_t acc_full, acc_empty;
+  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t drain, never;
 };
 
@@ -168,20 +174,17 @@ struct KvUnit {
   int32_t n, b, g, c;   // key tile, batch, kv head, d chunk
 };
 
-__device__ __forceinline__ int bwd_unit_index(int k, int n_units) {
-  const int grid = int(gridDim.x);
-  const int idx = k * grid + ((k & 1) ? (grid - 1 - int(blockIdx.x)) : int(blockIdx.x));
-  return idx < n_units ? idx : -1;
-}
-
-// Units in order of key tile n (most work first), then b, g, d chunk.
-__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int B, int Hkv, int NC) {
+// Units are claimed dynamically in the order (b, kv head g, key tile n, d chunk c):
+// CTAs busy at the same time work on one head group, sharing its Q / dO stream and
+// its dQ accumulator rows in L2; within a group n ascends, i.e. the work per unit
+// (the number of q tiles that see key tile n) descends, so each group ends with its
+// shortest units.
+__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int Hkv, int NT, int NC) {
   KvUnit u;
-  u.n = idx / (B * Hkv * NC);
-  const int rem = idx % (B * Hkv * NC);
-  u.b = rem / (Hkv * NC);
-  u.g = (rem / NC) % Hkv;
-  u.c = rem % NC;
+  u.c = idx % NC;
+  u.n = (idx / NC) % NT;
+  u.g = (idx / (NC * NT)) % Hkv;
+  u.b = idx / (NC * NT * Hkv);
   return u;
 }
 
@@ -248,6 +251,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
   __shared__ BwdBars bars;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ int unit_ring[kUnitRing];
 
   const int warp = int(warp_id()), lane = int(lane_id());
   if (threadIdx.x == 0) {
@@ -269,6 +273,10 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
     mbar_init(&bars.dq_empty, 4);
     mbar_init(&bars.acc_full, 1);
     mbar_init(&bars.acc_empty, 8);
+    for (int s = 0; s < kUnitRing; ++s) {
+      mbar_init(&bars.unit_full[s], 1);
+      mbar_init(&bars.unit_empty[s], 1 + 8 + 4);   // MMA thread + compute + dQ warps
+    }
     mbar_init(&bars.drain, 1);
     mbar_init(&bars.never, 1);
     fence_mbar_init();
@@ -297,9 +305,16 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
       uint32_t q_fills[2] = {0, 0};
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int idx = bwd_unit_index(k, prm.n_units);
+        // claim the next unit and hand it to the other roles through the ring
+        const int slot = k % kUnitRing;
+        if (k >= kUnitRing) ok = mbar_wait(&bars.unit_empty[slot], ((k / kUnitRing) - 1) & 1, wctx);
+        if (!ok) break;
+        int idx = atomicAdd(prm.counter, 1);
+        if (idx >= prm.n_units) idx = -1;
+        unit_ring[slot] = idx;
+        mbar_arrive(&bars.unit_full[slot]);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
         if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
@@ -396,9 +411,13 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
                    idesc_s, (kb | ks) != 0);
       };
       for (int k = 0; ok; ++k) {
-        const int idx = bwd_unit_index(k, prm.n_units);
+        const int slot = k % kUnitRing;
+        ok = mbar_wait(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+        if (!ok) break;
+        const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+        mbar_arrive(&bars.unit_empty[slot]);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
         const uint32_t cq = uint32_t(u.c * CB * BQ * 128);   // chunk offset in a Q / dO tile
         const uint32_t ck = uint32_t(u.c * CB * BKV * 128);  // chunk offset in the K tile
         ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
@@ -512,9 +531,14 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
     uint32_t dq_ph = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = bwd_unit_index(k, prm.n_units);
+      const int slot = k % kUnitRing;
+      ok = warp_wait_b(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+      if (!ok) break;
+      const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
       if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
+      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
       SlotWalk w;
       for (bool more = walk_first(prm, u.n, w); more; more = walk_next(prm, u.n, w)) {
         ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
@@ -555,9 +579,14 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
     uint32_t dsm_uses[2] = {0, 0};
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int idx = bwd_unit_index(k, prm.n_units);
+      const int slot = k % kUnitRing;
+      ok = warp_wait_b(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+      if (!ok) break;
+      const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
       if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.B, prm.Hkv, Cfg::NCHUNK);
+      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
       const int64_t key = int64_t(u.n) * BKV + row;
       SlotWalk w;
       int j = 0;
@@ -737,6 +766,8 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.n_qtiles = int32_t(twoC / Cfg::BQ);
   p.n_chunks = Cfg::NCHUNK;
   p.bq = Cfg::BQ;
+  p.n_ktiles = int32_t(a.S / Cfg::BKV);
+  p.counter = a.status + 32;
   p.scale = a.scale;
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
   p.status = a.status;
