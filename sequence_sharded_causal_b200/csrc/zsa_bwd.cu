@@ -28,6 +28,8 @@
 //    (TMEM -> fp32 reductions into the dQ accumulator), 1 TMA producer, 1 MMA issuer.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "zsa_kernels.h"
 #include "zsa_ptx.cuh"
 #include "zsa_tma_host.h"
@@ -203,7 +205,8 @@ __device__ __forceinline__ int64_t zz_pos(int64_t C, int32_t D, int32_t r, int64
 __device__ __forceinline__ bool tile_sees(const BwdParams& p, int32_t r, int32_t i, int32_t n,
                                           int64_t* p0) {
   *p0 = zz_pos(p.C, p.D, r, int64_t(i) * p.bq);
-  return !p.causal || (*p0 + p.bq - 1 >= int64_t(n) * 128);
+  // positions rise along a shard, so the tile's last row holds its largest position
+  return !p.causal || (zz_pos(p.C, p.D, r, int64_t(i) * p.bq + p.bq - 1) >= int64_t(n) * 128);
 }
 
 // First slot at or after (r, i, 0); false when the walk is over.
@@ -708,6 +711,469 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
   if (warp == Cfg::WARP_MMA) tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
+// ------------------------------------------------------------------ K3 for d <= 128
+// 128-row q slots, so every MMA of the slot is N = 128 (the tensor core loses most of
+// its rate on N = 64 shapes whose operands all come from shared memory).  TMEM holds
+// dV | dK | ST | XT: ST receives S^T and then the bf16 P^T and dS^T (half its columns
+// each, A operands of dV and dK); XT receives dP^T and, once the compute warps have
+// loaded it, dQ^T.  One slot is in flight; the next slot's S^T is issued as soon as
+// dK has consumed ST, its dP^T as soon as the dQ warps have read XT.
+template <int HD>
+struct BwdWideCfg {
+  static constexpr int BKV = 128;
+  static constexpr int BQ = 128;
+  static constexpr int KB = HD / 64;
+  static constexpr int NQST = 2;
+  static constexpr int KV_BYTES = BKV * HD * 2;
+  static constexpr int QT_BYTES = BQ * HD * 2;
+  static constexpr int DS_BYTES = BKV * BQ * 2;     // [2 q blocks][128 keys][64 q], 128B swizzle
+  static constexpr int SMEM_K = 0;
+  static constexpr int SMEM_V = SMEM_K + KV_BYTES;
+  static constexpr int SMEM_Q = SMEM_V + KV_BYTES;
+  static constexpr int SMEM_DO = SMEM_Q + NQST * QT_BYTES;
+  static constexpr int SMEM_DS = SMEM_DO + NQST * QT_BYTES;
+  static constexpr int SMEM_LSE = SMEM_DS + DS_BYTES;
+  static constexpr int SMEM_DELTA = SMEM_LSE + NQST * BQ * 4;
+  static constexpr int SMEM_BYTES = SMEM_DELTA + NQST * BQ * 4;
+  static constexpr int WARP_DQ = 8;
+  static constexpr int WARP_LOAD = 12;
+  static constexpr int WARP_MMA = 13;
+  static constexpr int NTHREADS = 14 * 32;
+  static constexpr uint32_t TM_DV = 0;
+  static constexpr uint32_t TM_DK = HD;
+  static constexpr uint32_t TM_ST = 2 * HD;
+  static constexpr uint32_t TM_XT = 2 * HD + BQ;
+  static constexpr uint32_t TM_COLS = 512;
+  static_assert(2 * HD + 2 * BQ <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+struct BwdWideBars {
+  uint64_t kv_full, kv_empty;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full, p_full, dp_full, ds_full;
+  uint64_t st_free, dsm_free, dq_full, dq_empty;
+  uint64_t acc_full, acc_empty;
+  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
+  uint64_t drain, never;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
+    zsa_bwd_wide_kernel(const __grid_constant__ CUtensorMap map_q,
+                        const __grid_constant__ CUtensorMap map_k,
+                        const __grid_constant__ CUtensorMap map_v,
+                        const __grid_constant__ CUtensorMap map_do, const BwdParams prm) {
+  using Cfg = BwdWideCfg<HD>;
+  constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV;
+  // the 128B-swizzled operand tiles need a 1024-byte aligned base; the shared-memory
+  // budget leaves no slack for aligning by hand, so the array itself is aligned
+  extern __shared__ __align__(1024) uint8_t smem_w[];
+  uint8_t* smem = smem_w;
+  __shared__ BwdWideBars bars;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  __shared__ int unit_ring[kUnitRing];
+
+  const int warp = int(warp_id()), lane = int(lane_id());
+  if (smem_u32(smem) & 1023u) {          // never expected; refuse rather than misread tiles
+    if (threadIdx.x == 0) atomicOr(prm.status, kDevTimeout);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    mbar_init(&bars.kv_full, 1);
+    mbar_init(&bars.kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_empty[s], 1 + 8);   // MMA commit + 8 compute warps
+    }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.p_full, 8);
+    mbar_init(&bars.dp_full, 1);
+    mbar_init(&bars.ds_full, 8);
+    mbar_init(&bars.st_free, 1);
+    mbar_init(&bars.dsm_free, 1);
+    mbar_init(&bars.dq_full, 1);
+    mbar_init(&bars.dq_empty, 4);
+    mbar_init(&bars.acc_full, 1);
+    mbar_init(&bars.acc_empty, 8);
+    for (int s = 0; s < kUnitRing; ++s) {
+      mbar_init(&bars.unit_full[s], 1);
+      mbar_init(&bars.unit_empty[s], 1 + 8 + 4);
+    }
+    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.never, 1);
+    fence_mbar_init();
+  }
+  if (warp == Cfg::WARP_MMA) {
+    tmem_alloc(&tmem_base_s, Cfg::TM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == Cfg::WARP_LOAD && lane == 0) {
+    tma_prefetch_desc(&map_q);
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_v);
+    tma_prefetch_desc(&map_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  const WaitCtx wctx{&abort_s, prm.status, prm.wait_limit_ns};
+  const int64_t twoC = 2 * prm.C;
+
+  if (warp == Cfg::WARP_LOAD) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t q_it = 0, kv_fills = 0;
+      uint32_t q_fills[2] = {0, 0};
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kUnitRing;
+        if (k >= kUnitRing) ok = mbar_wait(&bars.unit_empty[slot], ((k / kUnitRing) - 1) & 1, wctx);
+        if (!ok) break;
+        int idx = atomicAdd(prm.counter, 1);
+        if (idx >= prm.n_units) idx = -1;
+        unit_ring[slot] = idx;
+        mbar_arrive(&bars.unit_full[slot]);
+        if (idx < 0) break;
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+        if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
+        if (!ok) break;
+        mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
+        const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(u.n) * BKV);
+        for (int kb = 0; kb < KB; ++kb) {
+          tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128, &map_k, &bars.kv_full, kb * 64, u.g, key0);
+          tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128, &map_v, &bars.kv_full, kb * 64, u.g, key0);
+        }
+        ++kv_fills;
+        SlotWalk w;
+        for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
+          const int st = int(q_it & 1);
+          const uint32_t use = q_it >> 1;
+          if (use > 0) ok = mbar_wait(&bars.q_empty[st], (use - 1) & 1, wctx);
+          if (!ok) break;
+          const int32_t h = u.g * prm.G + w.e;
+          const int64_t rb = int64_t(w.r) * prm.B + u.b;
+          const int32_t row0 = int32_t(rb * twoC + int64_t(w.i) * BQ);
+          mbar_expect_tx(&bars.q_full[st], 2 * Cfg::QT_BYTES + 2 * BQ * 4);
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d(smem + Cfg::SMEM_Q + st * Cfg::QT_BYTES + kb * BQ * 128, &map_q,
+                        &bars.q_full[st], kb * 64, h, row0);
+            tma_load_3d(smem + Cfg::SMEM_DO + st * Cfg::QT_BYTES + kb * BQ * 128, &map_do,
+                        &bars.q_full[st], kb * 64, h, row0);
+          }
+          const int64_t stat = (rb * prm.Hq + h) * twoC + int64_t(w.i) * BQ;
+          bulk_load(smem + Cfg::SMEM_LSE + st * BQ * 4, prm.lse + stat, BQ * 4, &bars.q_full[st]);
+          bulk_load(smem + Cfg::SMEM_DELTA + st * BQ * 4, prm.delta + stat, BQ * 4, &bars.q_full[st]);
+          ++q_fills[st];
+          ++q_it;
+        }
+      }
+      if (!ok) {
+        const uint64_t lim = 1000000000ull;
+        if (kv_fills > 0) mbar_drain(&bars.kv_full, (kv_fills - 1) & 1, lim);
+        for (int s = 0; s < 2; ++s)
+          if (q_fills[s] > 0) mbar_drain(&bars.q_full[s], (q_fills[s] - 1) & 1, lim);
+      }
+    }
+  } else if (warp == Cfg::WARP_MMA) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
+      const uint32_t idesc_kv = idesc_bf16(128, HD, false, true);   // dV, dK (A from TMEM)
+      const uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);    // dQ^T
+      const uint32_t sK = smem_u32(smem + Cfg::SMEM_K);
+      const uint32_t sV = smem_u32(smem + Cfg::SMEM_V);
+      const uint32_t sQ = smem_u32(smem + Cfg::SMEM_Q);
+      const uint32_t sDO = smem_u32(smem + Cfg::SMEM_DO);
+      const uint32_t sDS = smem_u32(smem + Cfg::SMEM_DS);
+      // dQ^T = K^T dS^T: A = K^T (M = d in 64-row blocks at the K tile's d-block stride;
+      // with d = 64 the second M block reads V and its rows are never used)
+      const uint32_t lbo_kt = HD >= 128 ? uint32_t(BKV * 128) : uint32_t(Cfg::SMEM_V - Cfg::SMEM_K);
+      uint32_t kv_ph = 0, q_it = 0, p_ph = 0, ds_ph = 0;
+      uint32_t q_full_uses[2] = {0, 0};
+      uint32_t st_commits = 0, st_waits = 0, xt_commits = 0, xt_waits = 0, acc_commits = 0;
+      bool ok = true;
+      if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
+      // bf16 column of q rows 16ks .. 16ks+15 of P^T in ST: compute group h holds q rows
+      // 64h .. 64h+63 as 32 packed columns at 64h (dS^T at 64h + 32)
+      auto p_col = [](int ks) -> uint32_t { return uint32_t((ks >> 2) * 64 + (ks & 3) * 8); };
+      auto launch_slot = [&](int st) {          // S^T into ST, dP^T into XT
+        ok = ok && mbar_wait(&bars.q_full[st], q_full_uses[st] & 1, wctx);
+        ++q_full_uses[st];
+        if (ok && st_commits > st_waits) {
+          ok = mbar_wait(&bars.st_free, st_waits & 1, wctx);
+          ++st_waits;
+        }
+        if (!ok) return;
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + Cfg::TM_ST, sdesc_sw128(sK + kb * BKV * 128 + ks * 32, 16, 1024),
+                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
+                   idesc_s, (kb | ks) != 0);
+        mma_commit(&bars.s_full);
+        if (xt_commits > xt_waits) {
+          ok = mbar_wait(&bars.dq_empty, xt_waits & 1, wctx);
+          ++xt_waits;
+        }
+        if (!ok) return;
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sV + kb * BKV * 128 + ks * 32, 16, 1024),
+                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
+                   idesc_s, (kb | ks) != 0);
+        mma_commit(&bars.dp_full);
+      };
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kUnitRing;
+        ok = mbar_wait(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+        if (!ok) break;
+        const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+        mbar_arrive(&bars.unit_empty[slot]);
+        if (idx < 0) break;
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+        ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
+        kv_ph ^= 1;
+        if (!ok) break;
+        SlotWalk w;
+        bool more = walk_first(prm, u.n, w);
+        if (more) launch_slot(int(q_it & 1));
+        for (int j = 0; more && ok; ++j) {
+          const int st = int(q_it & 1);
+          SlotWalk nx = w;
+          const bool has_next = walk_next(prm, u.n, nx);
+          // dV += P^T dO
+          ok = mbar_wait(&bars.p_full, p_ph, wctx);
+          p_ph ^= 1;
+          if (ok && j == 0 && acc_commits > 0)
+            ok = mbar_wait(&bars.acc_empty, (acc_commits - 1) & 1, wctx);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BQ / 16; ++ks)
+            mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + p_col(ks),
+                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+                   (j > 0) || (ks > 0));
+          // dK += dS^T Q, then dQ^T = K^T dS^T into XT (dP^T there was loaded already)
+          ok = mbar_wait(&bars.ds_full, ds_ph, wctx);
+          ds_ph ^= 1;
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BQ / 16; ++ks)
+            mma_ts(tmem + Cfg::TM_DK, tmem + Cfg::TM_ST + p_col(ks) + 32,
+                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+                   (j > 0) || (ks > 0));
+          mma_commit(&bars.st_free);
+          ++st_commits;
+#pragma unroll
+          for (int ks = 0; ks < BKV / 16; ++ks)
+            mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sK + ks * 2048, lbo_kt, 1024),
+                   sdesc_sw128(sDS + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
+          mma_commit(&bars.dq_full);
+          ++xt_commits;
+          mma_commit(&bars.dsm_free);
+          mma_commit(&bars.q_empty[st]);
+          ++q_it;
+          if (has_next) launch_slot(int(q_it & 1));
+          w = nx;
+          more = has_next;
+        }
+        if (!ok) break;
+        mma_commit(&bars.acc_full);
+        ++acc_commits;
+        mma_commit(&bars.kv_empty);
+      }
+      mma_commit(&bars.drain);
+      mbar_drain(&bars.drain, 0, 1000000000ull);
+    }
+    __syncwarp();
+  } else if (warp >= Cfg::WARP_DQ) {
+    // ------------------------------------------------------------ dQ warps
+    const int qw = warp - Cfg::WARP_DQ;
+    const int drow = qw * 32 + lane;           // TMEM lane = d index of dQ^T
+    const uint32_t tXT = tmem + Cfg::TM_XT + (uint32_t(qw * 32) << 16);
+    uint32_t dq_ph = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int slot = k % kUnitRing;
+      ok = warp_wait_b(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+      if (!ok) break;
+      const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
+      if (idx < 0) break;
+      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+      SlotWalk w;
+      for (bool more = walk_first(prm, u.n, w); more; more = walk_next(prm, u.n, w)) {
+        ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
+        dq_ph ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        const int32_t h = u.g * prm.G + w.e;
+        const int64_t row0 = (int64_t(w.r) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
+        float* base = prm.dq_acc + (row0 * prm.Hq + h) * HD + drow;
+        const int64_t rstride = int64_t(prm.Hq) * HD;
+#pragma unroll 1
+        for (int t = 0; t < BQ / 32; t += 2) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tXT + t * 32, v0);
+          tmem_ld32(tXT + (t + 1) * 32, v1);
+          tmem_ld_wait();
+          if (t + 2 == BQ / 32) {          // all of dQ^T read: XT may be overwritten
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.dq_empty);
+          }
+          if (drow < HD) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) atomicAdd(base + (t * 32 + c) * rstride, __uint_as_float(v0[c]));
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              atomicAdd(base + ((t + 1) * 32 + c) * rstride, __uint_as_float(v1[c]));
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ compute warps
+    // group h = warp / 4 handles q rows 64h .. 64h+63 of every slot (contiguous
+    // positions: a 64-row half never straddles a zigzag chunk); thread = key row
+    const int hgrp = warp / 4;
+    const int qw = warp % 4;
+    const int row = qw * 32 + lane;
+    const uint32_t lane_addr = uint32_t(qw * 32) << 16;
+    const uint32_t tS = tmem + Cfg::TM_ST + 64 * hgrp + lane_addr;
+    const uint32_t tX = tmem + Cfg::TM_XT + 64 * hgrp + lane_addr;
+    uint8_t* dsb = smem + Cfg::SMEM_DS + hgrp * (BKV * 128);
+    uint32_t q_it = 0, s_ph = 0, dp_ph = 0, acc_ph = 0, dsm_uses = 0;
+    uint32_t q_full_uses[2] = {0, 0};
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int slot = k % kUnitRing;
+      ok = warp_wait_b(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
+      if (!ok) break;
+      const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
+      if (idx < 0) break;
+      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+      const int64_t key = int64_t(u.n) * BKV + row;
+      SlotWalk w;
+      for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
+        const int st = int(q_it & 1);
+        ok = warp_wait_b(&bars.q_full[st], q_full_uses[st] & 1, wctx);
+        ++q_full_uses[st];
+        if (!ok) break;
+        const float* lse_c = reinterpret_cast<const float*>(smem + Cfg::SMEM_LSE) + st * BQ + 64 * hgrp;
+        const float* dlt_c = reinterpret_cast<const float*>(smem + Cfg::SMEM_DELTA) + st * BQ + 64 * hgrp;
+        const int64_t p0 = zz_pos(prm.C, prm.D, w.r, int64_t(w.i) * BQ + 64 * hgrp);
+        const int nvis_lo = prm.causal ? int(key - p0) : 0;   // columns c < nvis_lo are masked
+        // ---- P^T = exp(scale S^T - lse) -> bf16 over the first half of this group's columns
+        ok = warp_wait_b(&bars.s_full, s_ph, wctx);
+        s_ph ^= 1;
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t pk[2][16];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sv[32];
+          tmem_ld32(tS + cc * 32, sv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = cc * 32 + 2 * e;
+            const float x0 = fmaf(__uint_as_float(sv[2 * e]), prm.scale_log2, -lse_c[c0] * kLog2e);
+            const float x1 = fmaf(__uint_as_float(sv[2 * e + 1]), prm.scale_log2, -lse_c[c0 + 1] * kLog2e);
+            pk[cc][e] = pack_bf16x2(c0 < nvis_lo ? 0.f : ex2_approx(x0),
+                                    c0 + 1 < nvis_lo ? 0.f : ex2_approx(x1));
+          }
+          tmem_st16(tS + cc * 16, pk[cc]);     // S^T columns already loaded
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full);
+        // ---- dS^T = P^T (dP^T - Delta) -> bf16 into the second half of the columns and
+        //      into shared memory (B operand of dQ^T)
+        ok = warp_wait_b(&bars.dp_full, dp_ph, wctx);
+        dp_ph ^= 1;
+        if (ok && dsm_uses > 0) ok = warp_wait_b(&bars.dsm_free, (dsm_uses - 1) & 1, wctx);
+        if (!ok) break;
+        ++dsm_uses;
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t sv[32];
+          tmem_ld32(tX + cc * 32, sv);
+          tmem_ld_wait();
+          uint32_t dk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = cc * 32 + 2 * e;
+            const float p0f = __uint_as_float(pk[cc][e] << 16);
+            const float p1f = __uint_as_float(pk[cc][e] & 0xFFFF0000u);
+            dk[e] = pack_bf16x2(p0f * (__uint_as_float(sv[2 * e]) - dlt_c[c0]),
+                                p1f * (__uint_as_float(sv[2 * e + 1]) - dlt_c[c0 + 1]));
+          }
+          tmem_st16(tS + 32 + cc * 16, dk);
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            *reinterpret_cast<uint4*>(dsb + sw128_offset(uint32_t(row), uint32_t(4 * cc + m))) =
+                make_uint4(dk[4 * m], dk[4 * m + 1], dk[4 * m + 2], dk[4 * m + 3]);
+        }
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars.ds_full);
+          mbar_arrive(&bars.q_empty[st]);     // lse / Delta of this stage consumed
+        }
+        ++q_it;
+      }
+      if (!ok) break;
+      // ---- epilogue: dV (group 0) / dK (group 1) rows of this key tile
+      ok = warp_wait_b(&bars.acc_full, acc_ph, wctx);
+      acc_ph ^= 1;
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tAcc = tmem + (hgrp == 0 ? Cfg::TM_DV : Cfg::TM_DK) + lane_addr;
+      const float mul = hgrp == 0 ? 1.0f : prm.scale;
+      __nv_bfloat16* dst = (hgrp == 0 ? prm.dv : prm.dk) +
+                           ((int64_t(u.b) * prm.S + key) * prm.Hkv + u.g) * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tAcc + c * 32, a);
+        tmem_ld_wait();
+        uint32_t o16[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          o16[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * mul, __uint_as_float(a[2 * e + 1]) * mul);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          d4[v4] = make_uint4(o16[4 * v4], o16[4 * v4 + 1], o16[4 * v4 + 2], o16[4 * v4 + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == Cfg::WARP_MMA) tmem_dealloc(tmem, Cfg::TM_COLS);
+}
+
 int num_sms() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -717,7 +1183,12 @@ int num_sms() {
 
 template <int HD>
 int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
-  using Cfg = BwdCfg<HD>;
+  // d <= 128: 128-row q slots (all MMAs N = 128); d = 256: 32-row slots over two d chunks
+  constexpr bool kWide = HD <= 128;
+  using Cfg = std::conditional_t<kWide, BwdWideCfg<HD>, BwdCfg<HD>>;
+  constexpr int kChunks = kWide ? 1 : HD / 128;    // d chunks of 128 per key tile
+  // the 128-row kernel aligns its dynamic shared memory itself (no slack needed)
+  constexpr int kSmem = kWide ? Cfg::SMEM_BYTES : Cfg::SMEM_BYTES + 1024;
   const int64_t rows = a.S * a.B;             // shard-major rows (D * B * 2C)
   const int64_t twoC = a.S / a.D;
   const int sms = num_sms();
@@ -762,9 +1233,9 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.S = a.S;
   p.C = a.S / (2 * int64_t(a.D));
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = a.Hq / a.Hkv; p.D = a.D; p.causal = a.causal;
-  p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / Cfg::BKV) * Cfg::NCHUNK);
+  p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / Cfg::BKV) * kChunks);
   p.n_qtiles = int32_t(twoC / Cfg::BQ);
-  p.n_chunks = Cfg::NCHUNK;
+  p.n_chunks = kChunks;
   p.bq = Cfg::BQ;
   p.n_ktiles = int32_t(a.S / Cfg::BKV);
   p.counter = a.status + 32;
@@ -773,17 +1244,21 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
   p.inject_stall = a.inject_stall;
-  const int smem = Cfg::SMEM_BYTES + 1024;
+  const int smem = kSmem;
+  auto kernel = [] {
+    if constexpr (kWide) return zsa_bwd_wide_kernel<HD>;
+    else return zsa_bwd_kernel<HD>;
+  }();
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(zsa_bwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return int(e);
     attr_set = true;
   }
   const int grid = p.n_units < sms ? p.n_units : sms;
   const TraceEvents tr = trace_events(2);
   if (tr.begin) cudaEventRecord(tr.begin, stream);
-  zsa_bwd_kernel<HD><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, p);
+  kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, p);
   cudaError_t e = cudaGetLastError();
   if (tr.end) cudaEventRecord(tr.end, stream);
   if (e != cudaSuccess) return int(e);
