@@ -43,6 +43,9 @@ CONFIGS = {
                  desc="long context: B=1 S=131072 Hq=32 Hkv=8 d=128 D=16, 0.1% Q/K rows x8"),
 }
 DEFAULT_CONFIG = "7b_mha"
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
+# the current kernel (profiles/); configurations without a capture report null.
+MEASURED_TRAFFIC = {("7b_mha", "zsa_bwd_wide_kernel"): 810018048 + 494552320}
 # Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
 CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
 
@@ -60,6 +63,21 @@ def load_peaks():
         return pk["bf16_tflops"], pk.get("bf16_tflops_sustained"), pk["hbm_gbs"], "measured"
     except Exception:
         return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def max_over_ranks(x, dist=None, device=None):
+    """The slowest rank's value (timing rule: max over ranks); x itself on one rank."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step, world, ms_max):
+    """Whole-job throughput: every rank's work per step over the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_max * 1e-3) / 1e12
 
 
 def dist_env():
@@ -256,10 +274,7 @@ def run_zsa(args, c, name):
     ms = e0.elapsed_time(e1) / K
     kms = [statistics.mean(kev[i][w][0].elapsed_time(kev[i][w][1]) for i in range(K))
            for w in range(4)]
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, dev)
 
     # ---- end to end through the API with host buffers (copies inside the timed region)
     pin = dict(pin_memory=True)
@@ -285,10 +300,8 @@ def run_zsa(args, c, name):
     x1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = x0.elapsed_time(x1) / K2
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
@@ -297,16 +310,17 @@ def run_zsa(args, c, name):
     peak, peak_sus, hbm, peak_src = load_peaks()
     ff = fwd_flops(c)
     bf = 2.5 * ff
-    value = world * (ff + bf) / (ms * 1e-3) / 1e12
+    value = job_tflops(ff + bf, world, ms)
     fwd_tf = ff / (kms[0] * 1e-3) / 1e12
     bwd_ms = kms[1] + kms[2] + kms[3]
     bwd_tf = bf / (bwd_ms * 1e-3) / 1e12
     main_tf = bf / (kms[2] * 1e-3) / 1e12
     # dominant kernel by time: forward kernel or backward main kernel
     if kms[2] >= kms[0]:
-        dom, dom_tf = "zsa_bwd_kernel", main_tf
+        dom, dom_tf = ("zsa_bwd_wide_kernel" if d <= 128 else "zsa_bwd_kernel"), main_tf
     else:
         dom, dom_tf = "zsa_fwd_kernel", fwd_tf
+    traffic = MEASURED_TRAFFIC.get((name, dom))
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -320,8 +334,8 @@ def run_zsa(args, c, name):
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": dom_tf, "peak": peak,
                      "unit": "TFLOP/s", "frac": dom_tf / peak, "peak_source": f"{peak_src} bf16 burst",
                      "frac_of_sustained": (dom_tf / peak_sus) if peak_sus else None,
-                     "traffic": None},
-        "e2e": {"value": world * (ff + bf) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                     "traffic": traffic},
+        "e2e": {"value": job_tflops(ff + bf, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
         "gpu_launches": 4 * K,
         "clocks": clk,

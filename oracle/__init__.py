@@ -44,6 +44,9 @@ def _load():
         lib.oracle_attn_fwd_rows.restype = ctypes.c_int
         lib.oracle_attn_bwd.argtypes = [i32, i64, i32, i32, i32, i32, i32, dbl] + [p] * 10
         lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_attn_dq_rows.argtypes = [i32, i64, i32, i32, i32, i32, i32, dbl, p, i64,
+                                            p, p, p, p, p]
+        lib.oracle_attn_dq_rows.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -134,6 +137,24 @@ def attn_fwd_rows(q_rows, rows, k, v, D, Hq, causal=True, scale=None):
     if rc != 0:
         raise ValueError("oracle_attn_fwd_rows: invalid problem")
     return o, lse
+
+
+def attn_dq_rows(q_rows, do_rows, rows, k, v, D, Hq, causal=True, scale=None):
+    """dQ of selected shard-major rows (rows as in attn_fwd_rows). Returns [n][Hq][d]."""
+    q_rows, do_rows, k, v = _f64(q_rows), _f64(do_rows), _f64(k), _f64(v)
+    rows = np.ascontiguousarray(np.asarray(rows, np.int64))
+    n = rows.shape[0]
+    B, S, Hkv, d = k.shape
+    assert q_rows.shape == (n, Hq, d) and do_rows.shape == (n, Hq, d)
+    if scale is None:
+        scale = float(np.float32(1.0 / np.sqrt(d)))
+    dq = np.empty((n, Hq, d), np.float64)
+    rc = _load().oracle_attn_dq_rows(B, S, Hq, Hkv, d, D, int(bool(causal)), float(scale),
+                                     _ptr(rows), n, _ptr(q_rows), _ptr(do_rows), _ptr(k), _ptr(v),
+                                     _ptr(dq))
+    if rc != 0:
+        raise ValueError("oracle_attn_dq_rows: invalid problem")
+    return dq
 
 
 def attn_bwd(q, k, v, dout, D, causal=True, scale=None):

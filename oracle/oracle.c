@@ -356,3 +356,54 @@ int oracle_attn_bwd(int32_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t d,
     }
     return 0;
 }
+
+/* dQ of selected shard-major rows only (each row's dQ needs nothing but its own q, dO
+ * and all of K, V: its forward is recomputed, Delta = <dO, O>, dS_k = P_k(dP_k -
+ * Delta), dQ = scale * sum_k dS_k k_k).
+ *   rows : [n] flattened (r*B + b)*2C + j;  q_rows, do_rows : [n][Hq][d]
+ *   dq_rows : [n][Hq][d] */
+int oracle_attn_dq_rows(int32_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t d,
+                        int32_t D, int32_t causal, double scale, const int64_t *rows,
+                        int64_t n, const double *q_rows, const double *do_rows,
+                        const double *k, const double *v, double *dq_rows)
+{
+    if (check_problem(B, S, Hq, Hkv, d, D)) return -1;
+    int64_t twoC = S / D;
+    int32_t G = Hq / Hkv;
+    for (int64_t x = 0; x < n; ++x)
+        if (rows[x] < 0 || rows[x] >= (int64_t)D * B * twoC) return -1;
+#pragma omp parallel
+    {
+        double *p_buf = (double *)malloc(sizeof(double) * (size_t)S);
+        double *o_row = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t idx = 0; idx < n * Hq; ++idx) {
+            int64_t x = idx / Hq;
+            int32_t h = (int32_t)(idx % Hq);
+            int64_t row = rows[x];
+            int32_t r = (int32_t)(row / ((int64_t)B * twoC));
+            int32_t b = (int32_t)((row / twoC) % B);
+            int64_t j = row % twoC;
+            int64_t p = zigzag_position(S, D, r, j);
+            int32_t kv = h / G;
+            const double *q_row = q_rows + (x * Hq + h) * d;
+            const double *do_row = do_rows + (x * Hq + h) * d;
+            double *dq_row = dq_rows + (x * Hq + h) * d;
+            int64_t nk;
+            attend_row(S, Hkv, d, causal, scale, q_row, p, k, v, b, kv, p_buf, o_row, &nk);
+            double dlt = 0.0;
+            for (int32_t t = 0; t < d; ++t) dlt += do_row[t] * o_row[t];
+            for (int32_t t = 0; t < d; ++t) dq_row[t] = 0.0;
+            for (int64_t key = 0; key < nk; ++key) {
+                int64_t kofs = (((int64_t)b * S + key) * Hkv + kv) * d;
+                double dp = 0.0;
+                for (int32_t t = 0; t < d; ++t) dp += do_row[t] * v[kofs + t];
+                double ds = p_buf[key] * (dp - dlt);
+                for (int32_t t = 0; t < d; ++t) dq_row[t] += scale * ds * k[kofs + t];
+            }
+        }
+        free(p_buf);
+        free(o_row);
+    }
+    return 0;
+}

@@ -56,18 +56,18 @@ bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 
 
 int check_sm100() {
   static std::mutex mu;
-  static std::map<int, int> verdict;
+  static std::map<int, int> arch_ok;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ZSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  auto it = verdict.find(dev);
-  if (it != verdict.end()) return it->second;
+  auto it = arch_ok.find(dev);
+  if (it != arch_ok.end()) return it->second;
   int major = 0, minor = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
     return ZSA_ERR_CUDA;
   int v = (major == 10 && minor == 0) ? ZSA_OK : ZSA_ERR_UNSUPPORTED;
-  verdict[dev] = v;
+  arch_ok[dev] = v;
   return v;
 }
 

@@ -311,6 +311,36 @@ def test_bwd_matches_matrix_form_every_D(oracle, S, Hq, Hkv, d):
         assert np.abs(_unshard_stats(g["delta"], perm) - delta).max() < 1e-11
 
 
+def test_dq_rows_match_full_backward(oracle):
+    rng = np.random.default_rng(13)
+    B, S, Hq, Hkv, d, D = 2, 64, 4, 2, 8, 4
+    q = _rand((D, B, S // D, Hq, d), rng)
+    do = _rand((D, B, S // D, Hq, d), rng)
+    k, v = _rand((B, S, Hkv, d), rng), _rand((B, S, Hkv, d), rng)
+    for causal in (True, False):
+        g = oracle.attn_bwd(q, k, v, do, D, causal)
+        rows = np.array([0, 3, 15, 16, 31, 40, 63, 64, 101, 127])
+        qf, dof = q.reshape(-1, Hq, d), do.reshape(-1, Hq, d)
+        dq = oracle.attn_dq_rows(qf[rows], dof[rows], rows, k, v, D, Hq, causal)
+        assert np.abs(dq - g["dq"].reshape(-1, Hq, d)[rows]).max() < 1e-13
+
+
+def test_gradient_identities(oracle):
+    # rows of P sum to 1 and rows of dS sum to 0, so per kv head
+    # sum_k dV_k = sum over the group's q rows of dO, and sum_k dK_k = 0
+    rng = np.random.default_rng(17)
+    B, S, Hq, Hkv, d, D = 1, 64, 4, 2, 8, 2
+    q = _rand((D, B, S // D, Hq, d), rng)
+    do = _rand((D, B, S // D, Hq, d), rng)
+    k, v = _rand((B, S, Hkv, d), rng), _rand((B, S, Hkv, d), rng)
+    g = oracle.attn_bwd(q, k, v, do, D)
+    G = Hq // Hkv
+    for kv in range(Hkv):
+        want = do[:, :, :, kv * G:(kv + 1) * G, :].sum(axis=(0, 2, 3))[0]
+        assert np.abs(g["dv"][0, :, kv].sum(0) - want).max() < 1e-12
+        assert np.abs(g["dk"][0, :, kv].sum(0)).max() < 1e-12
+
+
 def test_bwd_zero_upstream_gradient(oracle):
     rng = np.random.default_rng(9)
     B, S, Hq, Hkv, d, D = 1, 32, 2, 2, 8, 2
