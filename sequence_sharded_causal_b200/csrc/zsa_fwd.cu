@@ -14,15 +14,20 @@
 //    K/V tile fetched once feeds 2 x 128 rows of MMAs;
 //  * warp roles: 4 softmax warps per slot (one TMEM lane = one query row per thread),
 //    1 TMA producer warp, 1 MMA warp (one thread issues tcgen05.mma);
-//  * S = Q K^T goes to TMEM (128 x BK fp32); the softmax warps read it, apply the
-//    global-position mask, keep a running max (rescaling O in TMEM only when the max
-//    grows by more than 2^8) and write P as bf16 back over S; O += P V is a TMEM-A
-//    MMA (P from TMEM, V from shared memory as an MN-major operand);
+//  * S = Q K^T goes to one TMEM buffer (128 x BK fp32) shared by the slots; the softmax
+//    warps of the slot it belongs to copy it to registers and release it at once
+//    (s_free), apply the global-position mask, keep a running max (rescaling O in TMEM
+//    only when the max grows by more than 2^8) and write P as bf16 to the slot's own P
+//    columns; O += P V is a TMEM-A MMA (P from TMEM, V from shared memory as an
+//    MN-major operand);
 //  * shared memory: Q tiles resident for the unit, a K ring and a V ring of ST stages,
-//    all 128B-swizzled TMA tiles; TMEM: S0 | S1 | O0 | O1 (512 columns at d = 128).
-// MMA issue order per key tile n: PV0(n), QK0(n+1), PV1(n), QK1(n+1), so each slot's
-// softmax overlaps the other slot's two MMAs.  QK_s(n+1) overwrites the columns P_s(n)
-// lives in, so it is issued only after PV_s(n) has completed (pv_done barrier).
+//    all 128B-swizzled TMA tiles; TMEM: S | P0 | P1 | O0 | O1 (512 columns at d = 128).
+// The QK MMAs of a unit run in (key tile, slot) order through the S buffer, each one
+// issued as soon as the previous S has been copied out, so the next tile's scores are
+// computed while the softmax still works on the current one.  The MMA thread issues
+// PV_s(n) just before the QK whose S buffer slot s frees next (the softmax of slot s
+// reads S_s(n+1) right after publishing P_s(n)).  The softmax waits for PV_s(n-1)
+// (pv_done) only before it overwrites P_s or rescales O_s, after its exponentials.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -49,13 +54,15 @@ struct FwdCfg {
   static constexpr int SMEM_BYTES = SMEM_V + ST * KV_BYTES;
   static constexpr int NWARP_SOFTMAX = 4 * NSLOT;
   static constexpr int WARP_LOAD = NWARP_SOFTMAX;
-  static constexpr int WARP_MMA = NWARP_SOFTMAX + 1;
-  static constexpr int NTHREADS = (NWARP_SOFTMAX + 2) * 32;
+  static constexpr int WARP_MMA = NWARP_SOFTMAX + 1;   // QK issuer (and TMEM owner)
+  static constexpr int WARP_PV = NWARP_SOFTMAX + 2;    // PV issuer
+  static constexpr int NTHREADS = (NWARP_SOFTMAX + 3) * 32;
   static constexpr uint32_t TM_COLS = 512;
-  __device__ static constexpr uint32_t tm_s(int s) { return uint32_t(s * 128); }
+  static constexpr uint32_t TM_S = 0;                                     // BK columns
+  __device__ static constexpr uint32_t tm_p(int s) { return uint32_t(BK + s * (BK / 2)); }
   __device__ static constexpr uint32_t tm_o(int s) { return uint32_t(256 + s * HD); }
   static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
-  static_assert(256 + NSLOT * HD <= 512, "TMEM budget");
+  static_assert(BK + NSLOT * (BK / 2) <= 256 && 256 + NSLOT * HD <= 512, "TMEM budget");
 };
 
 struct FwdParams {
@@ -77,7 +84,7 @@ constexpr int kUnitRing = 4;  // claimed units in flight between the producer an
 struct FwdBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2], pv_done[2], o_full[2], o_empty[2];
+  uint64_t s_full[2], s_free, p_full[2], pv_done[2], o_full[2], o_empty[2];
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t drain;
   uint64_t never;  // test hook: no one ever arrives here
@@ -144,9 +151,10 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
     }
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&bars.unit_full[s], 1);
-      mbar_init(&bars.unit_empty[s], 1 + 4 * Cfg::NSLOT);   // MMA thread + softmax warps
+      mbar_init(&bars.unit_empty[s], 2 + 4 * Cfg::NSLOT);   // 2 MMA threads + softmax warps
     }
-    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.s_free, 4);                             // the 4 warps of the slot it held
+    mbar_init(&bars.drain, 2);                              // one commit per MMA thread
     mbar_init(&bars.never, 1);
     fence_mbar_init();
   }
@@ -201,25 +209,35 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
                         &bars.q_full[s], kb * 64, u.head[s], row0);
           ++q_fills[s];
         }
-        for (int n = 0; n < u.nmax && ok; ++n) {
-          const uint32_t it = kv_it + uint32_t(n);
-          const int st = int(it % ST);
-          const uint32_t use = it / ST;
-          const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(n) * BK);
-          if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, wctx);
-          if (!ok) break;
-          mbar_expect_tx(&bars.k_full[st], Cfg::KV_BYTES);
-          for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128, &map_k,
-                        &bars.k_full[st], kb * 64, u.g, key0);
-          ++k_fills[st];
-          if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, wctx);
-          if (!ok) break;
-          mbar_expect_tx(&bars.v_full[st], Cfg::KV_BYTES);
-          for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128, &map_v,
-                        &bars.v_full[st], kb * 64, u.g, key0);
-          ++v_fills[st];
+        // K runs one tile ahead of V: the MMA thread needs K(n+1) (for QK(n+1)) before
+        // V(n) (for PV(n)).
+        for (int n = 0; n <= u.nmax && ok; ++n) {
+          if (n < u.nmax) {
+            const uint32_t it = kv_it + uint32_t(n);
+            const int st = int(it % ST);
+            const uint32_t use = it / ST;
+            const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(n) * BK);
+            if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, wctx);
+            if (!ok) break;
+            mbar_expect_tx(&bars.k_full[st], Cfg::KV_BYTES);
+            for (int kb = 0; kb < KB; ++kb)
+              tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128, &map_k,
+                          &bars.k_full[st], kb * 64, u.g, key0);
+            ++k_fills[st];
+          }
+          if (n >= 1) {
+            const uint32_t it = kv_it + uint32_t(n - 1);
+            const int st = int(it % ST);
+            const uint32_t use = it / ST;
+            const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(n - 1) * BK);
+            if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, wctx);
+            if (!ok) break;
+            mbar_expect_tx(&bars.v_full[st], Cfg::KV_BYTES);
+            for (int kb = 0; kb < KB; ++kb)
+              tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128, &map_v,
+                          &bars.v_full[st], kb * 64, u.g, key0);
+            ++v_fills[st];
+          }
         }
         kv_it += uint32_t(u.nmax);
       }
@@ -234,32 +252,22 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         }
       }
     }
-  } else if (warp == Cfg::WARP_MMA) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == Cfg::WARP_MMA || warp == Cfg::WARP_PV) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads issue tcgen05.mma: one the QK list, one the PV list, each in (key tile
+    // n, slot s) order over the pairs with n < kend[s].  They share the tensor pipe but
+    // not their bookkeeping, so one thread's barrier waits and index arithmetic never
+    // leave the pipe idle while the other has work.  tcgen05.commit tracks the issuing
+    // thread's own MMAs, so each commits what it issued.
     if (lane == 0) {
+      const bool qk_role = warp == Cfg::WARP_MMA;
       const uint32_t idesc_qk = idesc_bf16(128, BK, false, false);
       const uint32_t idesc_pv = idesc_bf16(128, HD, false, true);
-      uint32_t kv_it = 0;
-      uint32_t q_ph[2] = {0, 0}, p_ph[2] = {0, 0}, pv_ph[2] = {0, 0}, oe_ph[2] = {0, 0};
-      bool pv_pending[2] = {false, false}, o_pending[2] = {false, false};
+      uint32_t kv_it = 0, qk_total = 0;
+      // per-slot phase bits (bit s), kept in registers: the slot index is dynamic here
+      uint32_t q_ph = 0, p_ph = 0, oe_ph = 0, o_pending = 0;
       bool ok = true;
       if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
-      auto issue_qk = [&](int s, int st) {
-        for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = sdesc_sw128(sQ + s * Cfg::Q_BYTES + kb * 128 * 128 + ks * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(sK + st * Cfg::KV_BYTES + kb * BK * 128 + ks * 32, 16, 1024);
-            mma_ss(tmem + Cfg::tm_s(s), a, b, idesc_qk, (kb | ks) != 0);
-          }
-      };
-      auto issue_pv = [&](int s, int st, int n) {
-#pragma unroll
-        for (int ks = 0; ks < BK / 16; ++ks) {
-          const uint64_t b = sdesc_sw128(sV + st * Cfg::KV_BYTES + ks * 2048, BK * 128, 1024);
-          mma_ts(tmem + Cfg::tm_o(s), tmem + Cfg::tm_s(s) + ks * 8, b, idesc_pv, (n > 0) || (ks > 0));
-        }
-      };
       for (int k = 0; ok; ++k) {
         const int slot = k % kUnitRing;
         ok = mbar_wait(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
@@ -268,75 +276,79 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         mbar_arrive(&bars.unit_empty[slot]);
         if (idx < 0) break;
         const UnitInfo u = load_unit(prm.units, idx);
-        for (int s = 0; s < NSLOT && ok; ++s) {
-          if (u.kend[s] == 0) continue;
-          ok = mbar_wait(&bars.q_full[s], q_ph[s], wctx);
-          q_ph[s] ^= 1;
-        }
-        if (!ok) break;
-        // prologue: S_s(0) = Q_s K(0)^T
-        {
-          const int st = int(kv_it % ST);
-          ok = mbar_wait(&bars.k_full[st], (kv_it / ST) & 1, wctx);
-          if (!ok) break;
+        const int k0 = u.kend[0], k1 = NSLOT == 2 ? u.kend[1] : 0;
+        // (n, s) walk over present pairs; first / last: s opens / closes key tile n
+        int n = 0, sl = k0 > 0 ? 0 : 1;
+        if (qk_role) {
           for (int s = 0; s < NSLOT && ok; ++s) {
             if (u.kend[s] == 0) continue;
-            if (pv_pending[s]) {
-              ok = mbar_wait(&bars.pv_done[s], pv_ph[s], wctx);
-              pv_ph[s] ^= 1;
-              pv_pending[s] = false;
-              if (!ok) break;
-            }
-            tc_fence_after();
-            issue_qk(s, st);
-            mma_commit(&bars.s_full[s]);
-            if (u.kend[s] == 1) mma_commit(&bars.q_empty[s]);
+            ok = mbar_wait(&bars.q_full[s], (q_ph >> s) & 1u, wctx);
+            q_ph ^= 1u << s;
           }
-          if (!ok) break;
-          mma_commit(&bars.k_empty[st]);
-        }
-        for (int n = 0; n < u.nmax && ok; ++n) {
-          const uint32_t it = kv_it + uint32_t(n);
-          const int st = int(it % ST);
-          const int st1 = int((it + 1) % ST);
-          ok = mbar_wait(&bars.v_full[st], (it / ST) & 1, wctx);
-          bool knext = false;
-          for (int s = 0; s < NSLOT && ok; ++s) {
-            if (n >= u.kend[s]) continue;
-            ok = mbar_wait(&bars.p_full[s], p_ph[s], wctx);
-            p_ph[s] ^= 1;
-            if (ok && n == 0 && o_pending[s]) {
-              ok = mbar_wait(&bars.o_empty[s], oe_ph[s], wctx);
-              oe_ph[s] ^= 1;
-              o_pending[s] = false;
+          for (int i = 0; i < k0 + k1 && ok; ++i) {
+            // ---- QK_sl(n): S = Q_sl K(n)^T into the shared S buffer
+            const uint32_t it = kv_it + uint32_t(n);
+            const int st = int(it % ST);
+            const bool first = sl == 0 || n >= k0;
+            const bool last = sl == 1 || n >= k1;
+            if (qk_total > 0) ok = mbar_wait(&bars.s_free, (qk_total - 1) & 1, wctx);
+            if (ok && first) ok = mbar_wait(&bars.k_full[st], (it / ST) & 1, wctx);
+            if (!ok) break;
+            tc_fence_after();
+            for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t a = sdesc_sw128(sQ + sl * Cfg::Q_BYTES + kb * 128 * 128 + ks * 32, 16, 1024);
+                const uint64_t b = sdesc_sw128(sK + st * Cfg::KV_BYTES + kb * BK * 128 + ks * 32, 16, 1024);
+                mma_ss(tmem + Cfg::TM_S, a, b, idesc_qk, (kb | ks) != 0);
+              }
+            mma_commit(&bars.s_full[sl]);
+            if (n == (sl == 0 ? k0 : k1) - 1) mma_commit(&bars.q_empty[sl]);
+            if (last) mma_commit(&bars.k_empty[st]);
+            ++qk_total;
+            if (sl == 0 && n < k1) {
+              sl = 1;
+            } else {
+              ++n;
+              sl = n < k0 ? 0 : 1;
+            }
+          }
+        } else {
+          for (int i = 0; i < k0 + k1 && ok; ++i) {
+            // ---- PV_sl(n): O_sl += P_sl V(n)
+            const uint32_t it = kv_it + uint32_t(n);
+            const int st = int(it % ST);
+            const bool first = sl == 0 || n >= k0;
+            const bool last = sl == 1 || n >= k1;
+            if (first) ok = mbar_wait(&bars.v_full[st], (it / ST) & 1, wctx);
+            if (ok) ok = mbar_wait(&bars.p_full[sl], (p_ph >> sl) & 1u, wctx);
+            p_ph ^= 1u << sl;
+            if (ok && n == 0 && ((o_pending >> sl) & 1u)) {
+              ok = mbar_wait(&bars.o_empty[sl], (oe_ph >> sl) & 1u, wctx);
+              oe_ph ^= 1u << sl;
+              o_pending &= ~(1u << sl);
             }
             if (!ok) break;
             tc_fence_after();
-            issue_pv(s, st, n);
-            mma_commit(&bars.pv_done[s]);
-            pv_pending[s] = true;
-            if (n == u.kend[s] - 1) {
-              mma_commit(&bars.o_full[s]);
-              o_pending[s] = true;
+            const uint32_t tO = tmem + Cfg::tm_o(sl), tP = tmem + Cfg::tm_p(sl);
+#pragma unroll
+            for (int ks = 0; ks < BK / 16; ++ks) {
+              const uint64_t b = sdesc_sw128(sV + st * Cfg::KV_BYTES + ks * 2048, BK * 128, 1024);
+              mma_ts(tO, tP + ks * 8, b, idesc_pv, (n > 0) || (ks > 0));
             }
-            if (n + 1 < u.kend[s]) {
-              if (!knext) {
-                ok = mbar_wait(&bars.k_full[st1], ((it + 1) / ST) & 1, wctx);
-                knext = true;
-              }
-              if (ok) ok = mbar_wait(&bars.pv_done[s], pv_ph[s], wctx);
-              pv_ph[s] ^= 1;
-              pv_pending[s] = false;
-              if (!ok) break;
-              tc_fence_after();
-              issue_qk(s, st1);
-              mma_commit(&bars.s_full[s]);
-              if (n + 1 == u.kend[s] - 1) mma_commit(&bars.q_empty[s]);
+            mma_commit(&bars.pv_done[sl]);
+            if (n == (sl == 0 ? k0 : k1) - 1) {
+              mma_commit(&bars.o_full[sl]);
+              o_pending |= 1u << sl;
+            }
+            if (last) mma_commit(&bars.v_empty[st]);
+            if (sl == 0 && n < k1) {
+              sl = 1;
+            } else {
+              ++n;
+              sl = n < k0 ? 0 : 1;
             }
           }
-          if (!ok) break;
-          mma_commit(&bars.v_empty[st]);
-          if (knext) mma_commit(&bars.k_empty[st1]);
         }
         kv_it += uint32_t(u.nmax);
       }
@@ -351,9 +363,11 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
     const int qw = warp % 4;           // TMEM lane quarter
     const int row = qw * 32 + lane;    // query row within the tile = TMEM lane
     const uint32_t lane_addr = uint32_t(qw * 32) << 16;
-    const uint32_t tS = tmem + Cfg::tm_s(s) + lane_addr;
+    const uint32_t tS = tmem + Cfg::TM_S + lane_addr;
+    const uint32_t tP = tmem + Cfg::tm_p(s) + lane_addr;
     const uint32_t tO = tmem + Cfg::tm_o(s) + lane_addr;
     uint32_t s_ph = 0, o_ph = 0;
+    uint32_t pv_base = 0;              // PV_s MMAs committed in earlier units
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int slot = k % kUnitRing;
@@ -378,6 +392,10 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
 #pragma unroll
         for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, sr[c]);
         tmem_ld_wait();
+        // the scores are in registers: the S buffer may take the next QK
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_free);
         // Causal mask on the tiles that cross this warp's diagonal only: keys past
         // `lim` (relative to the tile) are invisible to this row.  Off-diagonal tiles
         // (all but about one in kend) skip the mask entirely.
@@ -410,6 +428,36 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
           if (n > 0) alpha = ex2_approx(m_run - m_new);
           m_run = m_new;
         }
+        // P = 2^(s*scale*log2e - m), two elements per packed FMA.  Two row sums, in
+        // packed adds: of the fp32 P (for lse) and of the bf16-rounded P the PV MMA
+        // consumes (normalises O, keeping it a convex combination of V rows: exact when
+        // one key dominates a row).
+        const uint64_t scale2 = f2_pack(prm.scale_log2, prm.scale_log2);
+        const uint64_t negm2 = f2_pack(-m_run, -m_run);
+        uint64_t lsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        uint64_t rsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        uint32_t pk[BK / 32][16];
+#pragma unroll
+        for (int c = 0; c < BK / 32; ++c) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
+                                       scale2, negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            lsum2[e & 1] = f2_add(lsum2[e & 1], f2_pack(p0, p1));
+            pk[c][e] = pack_bf16x2(p0, p1);
+            rsum2[e & 1] = f2_add(rsum2[e & 1], bf16x2_widen(pk[c][e]));
+          }
+        }
+        // P_s and O_s are free once PV_s(n-1) has completed
+        if (n > 0) {
+          ok = warp_wait(&bars.pv_done[s], (pv_base + uint32_t(n) - 1) & 1, wctx);
+          if (!ok) break;
+          tc_fence_after();
+        }
         if (__any_sync(0xffffffffu, grow && n > 0)) {
           l_run *= alpha;
           r_run *= alpha;
@@ -423,31 +471,8 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             tmem_st32(tO + c * 32, orow);
           }
         }
-        // P = 2^(s*scale*log2e - m), two elements per packed FMA.  Two row sums, in
-        // packed adds: of the fp32 P (for lse) and of the bf16-rounded P the PV MMA
-        // consumes (normalises O, keeping it a convex combination of V rows: exact when
-        // one key dominates a row).
-        const uint64_t scale2 = f2_pack(prm.scale_log2, prm.scale_log2);
-        const uint64_t negm2 = f2_pack(-m_run, -m_run);
-        uint64_t lsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-        uint64_t rsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-        for (int c = 0; c < BK / 32; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])),
-                                       scale2, negm2);
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
-            lsum2[e & 1] = f2_add(lsum2[e & 1], f2_pack(p0, p1));
-            pk[e] = pack_bf16x2(p0, p1);
-            rsum2[e & 1] = f2_add(rsum2[e & 1], bf16x2_widen(pk[e]));
-          }
-          tmem_st16(tS + c * 16, pk);     // P (bf16 pairs) over the S columns already read
-        }
+        for (int c = 0; c < BK / 32; ++c) tmem_st16(tP + c * 16, pk[c]);
         float a0, a1, b0, b1;
         f2_unpack(f2_add(lsum2[0], lsum2[1]), a0, a1);
         f2_unpack(f2_add(rsum2[0], rsum2[1]), b0, b1);
@@ -459,6 +484,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         if (lane == 0) mbar_arrive(&bars.p_full[s]);
       }
       if (!ok) break;
+      pv_base += uint32_t(u.kend[s]);
       // ---- epilogue: O / l -> bf16, lse
       ok = warp_wait(&bars.o_full[s], o_ph, wctx);
       o_ph ^= 1;
