@@ -737,8 +737,9 @@ struct BwdWideCfg {
   static constexpr int SMEM_BYTES = SMEM_DELTA + NQST * BQ * 4;
   static constexpr int WARP_DQ = 8;
   static constexpr int WARP_LOAD = 12;
-  static constexpr int WARP_MMA = 13;
-  static constexpr int NTHREADS = 14 * 32;
+  static constexpr int WARP_MMA = 13;   // S^T, dP^T issuer (and TMEM owner)
+  static constexpr int WARP_MMA2 = 14;  // dV, dK, dQ^T issuer
+  static constexpr int NTHREADS = 15 * 32;
   static constexpr uint32_t TM_DV = 0;
   static constexpr uint32_t TM_DK = HD;
   static constexpr uint32_t TM_ST = 2 * HD;
@@ -800,9 +801,9 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     mbar_init(&bars.acc_empty, 8);
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&bars.unit_full[s], 1);
-      mbar_init(&bars.unit_empty[s], 1 + 8 + 4);
+      mbar_init(&bars.unit_empty[s], 2 + 8 + 4);   // 2 MMA threads + compute + dQ warps
     }
-    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.drain, 2);                     // one commit per MMA thread
     mbar_init(&bars.never, 1);
     fence_mbar_init();
   }
@@ -878,9 +879,18 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
           if (q_fills[s] > 0) mbar_drain(&bars.q_full[s], (q_fills[s] - 1) & 1, lim);
       }
     }
-  } else if (warp == Cfg::WARP_MMA) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == Cfg::WARP_MMA || warp == Cfg::WARP_MMA2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Thread A (WARP_MMA) issues each slot's S^T and dP^T, thread B (WARP_MMA2) its dV,
+    // dK and dQ^T.  Their TMEM hand-offs are barriers already (st_free: B's dK has
+    // consumed ST; dq_empty: the dQ warps have read XT; ds_full: the compute warps have
+    // read dP^T), so neither waits on the other's issue order, and one thread's barrier
+    // latency no longer idles the tensor pipe.  tcgen05.commit tracks the issuing
+    // thread's own MMAs: everything that needs both threads' MMAs finished (q_empty,
+    // kv_empty, acc_full) is committed by B, whose MMAs start only after A's of the same
+    // slot have completed (p_full / ds_full follow s_full / dp_full).
     if (lane == 0) {
+      const bool role_a = warp == Cfg::WARP_MMA;
       const uint32_t idesc_s = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
       const uint32_t idesc_kv = idesc_bf16(128, HD, false, true);   // dV, dK (A from TMEM)
       const uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);    // dQ^T
@@ -894,42 +904,12 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
       const uint32_t lbo_kt = HD >= 128 ? uint32_t(BKV * 128) : uint32_t(Cfg::SMEM_V - Cfg::SMEM_K);
       uint32_t kv_ph = 0, q_it = 0, p_ph = 0, ds_ph = 0;
       uint32_t q_full_uses[2] = {0, 0};
-      uint32_t st_commits = 0, st_waits = 0, xt_commits = 0, xt_waits = 0, acc_commits = 0;
+      uint32_t st_waits = 0, xt_waits = 0, acc_commits = 0;
       bool ok = true;
       if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
       // bf16 column of q rows 16ks .. 16ks+15 of P^T in ST: compute group h holds q rows
       // 64h .. 64h+63 as 32 packed columns at 64h (dS^T at 64h + 32)
       auto p_col = [](int ks) -> uint32_t { return uint32_t((ks >> 2) * 64 + (ks & 3) * 8); };
-      auto launch_slot = [&](int st) {          // S^T into ST, dP^T into XT
-        ok = ok && mbar_wait(&bars.q_full[st], q_full_uses[st] & 1, wctx);
-        ++q_full_uses[st];
-        if (ok && st_commits > st_waits) {
-          ok = mbar_wait(&bars.st_free, st_waits & 1, wctx);
-          ++st_waits;
-        }
-        if (!ok) return;
-        tc_fence_after();
-        for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + Cfg::TM_ST, sdesc_sw128(sK + kb * BKV * 128 + ks * 32, 16, 1024),
-                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
-                   idesc_s, (kb | ks) != 0);
-        mma_commit(&bars.s_full);
-        if (xt_commits > xt_waits) {
-          ok = mbar_wait(&bars.dq_empty, xt_waits & 1, wctx);
-          ++xt_waits;
-        }
-        if (!ok) return;
-        tc_fence_after();
-        for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sV + kb * BKV * 128 + ks * 32, 16, 1024),
-                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
-                   idesc_s, (kb | ks) != 0);
-        mma_commit(&bars.dp_full);
-      };
       for (int k = 0; ok; ++k) {
         const int slot = k % kUnitRing;
         ok = mbar_wait(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
@@ -938,57 +918,79 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         mbar_arrive(&bars.unit_empty[slot]);
         if (idx < 0) break;
         const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
-        ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
-        kv_ph ^= 1;
-        if (!ok) break;
+        if (role_a) {
+          ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
+          kv_ph ^= 1;
+          if (!ok) break;
+        }
         SlotWalk w;
-        bool more = walk_first(prm, u.n, w);
-        if (more) launch_slot(int(q_it & 1));
-        for (int j = 0; more && ok; ++j) {
+        for (bool more = walk_first(prm, u.n, w), j0 = true; more && ok;
+             more = walk_next(prm, u.n, w), j0 = false) {
           const int st = int(q_it & 1);
-          SlotWalk nx = w;
-          const bool has_next = walk_next(prm, u.n, nx);
-          // dV += P^T dO
-          ok = mbar_wait(&bars.p_full, p_ph, wctx);
-          p_ph ^= 1;
-          if (ok && j == 0 && acc_commits > 0)
-            ok = mbar_wait(&bars.acc_empty, (acc_commits - 1) & 1, wctx);
-          if (!ok) break;
-          tc_fence_after();
+          if (role_a) {
+            // S^T into ST once this stage's Q is in and B's dK has consumed ST
+            ok = mbar_wait(&bars.q_full[st], q_full_uses[st] & 1, wctx);
+            ++q_full_uses[st];
+            if (ok && q_it > 0) ok = mbar_wait(&bars.st_free, st_waits++ & 1, wctx);
+            if (!ok) break;
+            tc_fence_after();
+            for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-          for (int ks = 0; ks < BQ / 16; ++ks)
-            mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + p_col(ks),
-                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
-                   (j > 0) || (ks > 0));
-          // dK += dS^T Q, then dQ^T = K^T dS^T into XT (dP^T there was loaded already)
-          ok = mbar_wait(&bars.ds_full, ds_ph, wctx);
-          ds_ph ^= 1;
-          if (!ok) break;
-          tc_fence_after();
+              for (int ks = 0; ks < 4; ++ks)
+                mma_ss(tmem + Cfg::TM_ST, sdesc_sw128(sK + kb * BKV * 128 + ks * 32, 16, 1024),
+                       sdesc_sw128(sQ + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
+                       idesc_s, (kb | ks) != 0);
+            mma_commit(&bars.s_full);
+            // dP^T into XT once the dQ warps have read the previous dQ^T out of it
+            if (q_it > 0) ok = mbar_wait(&bars.dq_empty, xt_waits++ & 1, wctx);
+            if (!ok) break;
+            tc_fence_after();
+            for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-          for (int ks = 0; ks < BQ / 16; ++ks)
-            mma_ts(tmem + Cfg::TM_DK, tmem + Cfg::TM_ST + p_col(ks) + 32,
-                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
-                   (j > 0) || (ks > 0));
-          mma_commit(&bars.st_free);
-          ++st_commits;
+              for (int ks = 0; ks < 4; ++ks)
+                mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sV + kb * BKV * 128 + ks * 32, 16, 1024),
+                       sdesc_sw128(sDO + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
+                       idesc_s, (kb | ks) != 0);
+            mma_commit(&bars.dp_full);
+          } else {
+            // dV += P^T dO
+            ok = mbar_wait(&bars.p_full, p_ph, wctx);
+            p_ph ^= 1;
+            if (ok && j0 && acc_commits > 0) ok = mbar_wait(&bars.acc_empty, (acc_commits - 1) & 1, wctx);
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < BKV / 16; ++ks)
-            mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sK + ks * 2048, lbo_kt, 1024),
-                   sdesc_sw128(sDS + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
-          mma_commit(&bars.dq_full);
-          ++xt_commits;
-          mma_commit(&bars.dsm_free);
-          mma_commit(&bars.q_empty[st]);
+            for (int ks = 0; ks < BQ / 16; ++ks)
+              mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + p_col(ks),
+                     sdesc_sw128(sDO + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+                     !j0 || (ks > 0));
+            // dK += dS^T Q, then dQ^T = K^T dS^T into XT (dP^T there was loaded already)
+            ok = mbar_wait(&bars.ds_full, ds_ph, wctx);
+            ds_ph ^= 1;
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < BQ / 16; ++ks)
+              mma_ts(tmem + Cfg::TM_DK, tmem + Cfg::TM_ST + p_col(ks) + 32,
+                     sdesc_sw128(sQ + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
+                     !j0 || (ks > 0));
+            mma_commit(&bars.st_free);
+#pragma unroll
+            for (int ks = 0; ks < BKV / 16; ++ks)
+              mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sK + ks * 2048, lbo_kt, 1024),
+                     sdesc_sw128(sDS + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
+            mma_commit(&bars.dq_full);
+            mma_commit(&bars.dsm_free);
+            mma_commit(&bars.q_empty[st]);
+          }
           ++q_it;
-          if (has_next) launch_slot(int(q_it & 1));
-          w = nx;
-          more = has_next;
         }
         if (!ok) break;
-        mma_commit(&bars.acc_full);
-        ++acc_commits;
-        mma_commit(&bars.kv_empty);
+        if (!role_a) {
+          mma_commit(&bars.acc_full);
+          ++acc_commits;
+          mma_commit(&bars.kv_empty);
+        }
       }
       mma_commit(&bars.drain);
       mbar_drain(&bars.drain, 0, 1000000000ull);
