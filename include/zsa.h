@@ -116,7 +116,7 @@ ZSA_API int zsa_partition(const zsa_problem* problem, zsa_tiling* tiling, int32_
 /* Workspace bytes needed by zsa_attn_fwd (pass = 0) or zsa_attn_bwd (pass = 1).
  * The workspace must be device memory, 256-byte aligned, not shared between calls in
  * flight.  fwd: status word + the unit table.  bwd: status word + Delta (fp32
- * [D][B][Hq][2C]) + a dQ accumulator (fp32 [D][B][2C][Hq][d]). */
+ * [D][B][Hq][2C]) + a dQ accumulator (fp32, head-major [Hq][D*B*2C][d]). */
 ZSA_API int zsa_workspace_bytes(const zsa_problem* problem, int pass, size_t* bytes_out);
 
 /* Forward: o (bf16, Q layout) and lse (fp32 [D][B][Hq][2C]).  q, k, v, o, lse and the

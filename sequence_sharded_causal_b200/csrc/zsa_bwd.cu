@@ -67,6 +67,8 @@ __global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* _
         acc = fmaf(x.x, y.x, acc);
         acc = fmaf(x.y, y.y, acc);
       }
+      // zero d floats per (row, head) pair: the pairs tile the whole accumulator, so this
+      // holds for its head-major layout too
       float4* z = reinterpret_cast<float4*>(dq_acc + pair * HD) + 2 * sub;
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -83,19 +85,28 @@ __global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* _
 }
 
 // ------------------------------------------------------------------ K4: dQ = bf16(scale*acc)
+// The accumulator is head-major, [Hq][rows][d] (one q head's rows contiguous, so the
+// reductions of a 128-row slot land in one 64 KB block instead of 128 lines 16 KB
+// apart); dQ is [rows][Hq][d].  One block per row (grid-stride): each thread turns 8
+// consecutive fp32 of one head into one 16-byte bf16 store.
+template <int HD>
 __global__ void __launch_bounds__(256) zsa_dq_convert_kernel(const float* __restrict__ acc,
                                                              __nv_bfloat16* __restrict__ dq,
-                                                             int64_t n8, float scale) {
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += int64_t(gridDim.x) * blockDim.x) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
-    uint4 r;
-    r.x = pack_bf16x2(a.x * scale, a.y * scale);
-    r.y = pack_bf16x2(a.z * scale, a.w * scale);
-    r.z = pack_bf16x2(b.x * scale, b.y * scale);
-    r.w = pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[i] = r;
+                                                             int64_t rows, int32_t Hq, float scale) {
+  constexpr int V8 = HD / 8;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    for (int t = threadIdx.x; t < Hq * V8; t += blockDim.x) {
+      const int h = t / V8, d8 = t % V8;
+      const float4* src = reinterpret_cast<const float4*>(acc + (int64_t(h) * rows + row) * HD) + 2 * d8;
+      const float4 a = src[0];
+      const float4 b = src[1];
+      uint4 r;
+      r.x = pack_bf16x2(a.x * scale, a.y * scale);
+      r.y = pack_bf16x2(a.z * scale, a.w * scale);
+      r.z = pack_bf16x2(b.x * scale, b.y * scale);
+      r.w = pack_bf16x2(b.z * scale, b.w * scale);
+      reinterpret_cast<uint4*>(dq + row * int64_t(Hq) * HD)[t] = r;
+    }
   }
 }
 
@@ -558,8 +569,9 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
         if (drow < HC) {
           const int32_t h = u.g * prm.G + w.e;
           const int64_t row0 = (int64_t(w.r) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
-          float* base = prm.dq_acc + (row0 * prm.Hq + h) * HD + u.c * HC + drow;
-          const int64_t rstride = int64_t(prm.Hq) * HD;
+          // head-major accumulator [Hq][rows][d]
+          float* base = prm.dq_acc + (int64_t(h) * prm.B * prm.S + row0) * HD + u.c * HC + drow;
+          const int64_t rstride = HD;
 #pragma unroll
           for (int t = 0; t < BQ / 32; ++t)
 #pragma unroll
@@ -1020,8 +1032,9 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         tc_fence_after();
         const int32_t h = u.g * prm.G + w.e;
         const int64_t row0 = (int64_t(w.r) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
-        float* base = prm.dq_acc + (row0 * prm.Hq + h) * HD + drow;
-        const int64_t rstride = int64_t(prm.Hq) * HD;
+        // head-major accumulator [Hq][rows][d]: the slot's 128 rows are one 64 KB block
+        float* base = prm.dq_acc + (int64_t(h) * prm.B * prm.S + row0) * HD + drow;
+        const int64_t rstride = HD;
 #pragma unroll 1
         for (int t = 0; t < BQ / 32; t += 2) {
           uint32_t v0[32], v1[32];
@@ -1266,13 +1279,12 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return int(e);
   // K4
   {
-    const int64_t n8 = rows * a.Hq * HD / 8;
-    int64_t blocks = (n8 + 255) / 256;
+    int64_t blocks = rows;
     if (blocks > int64_t(sms) * 16) blocks = int64_t(sms) * 16;
     const TraceEvents tr4 = trace_events(3);
     if (tr4.begin) cudaEventRecord(tr4.begin, stream);
-    zsa_dq_convert_kernel<<<int(blocks), 256, 0, stream>>>(a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq),
-                                                            n8, a.scale);
+    zsa_dq_convert_kernel<HD><<<int(blocks), 256, 0, stream>>>(
+        a.dq_acc, reinterpret_cast<__nv_bfloat16*>(a.dq), rows, a.Hq, a.scale);
     e = cudaGetLastError();
     if (tr4.end) cudaEventRecord(tr4.end, stream);
   }

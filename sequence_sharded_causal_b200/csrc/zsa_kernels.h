@@ -34,7 +34,7 @@ struct BwdArgs {
   void* dk;
   void* dv;
   float* delta;            // [D][B][Hq][2C] workspace
-  float* dq_acc;           // [D][B][2C][Hq][d] workspace
+  float* dq_acc;           // [Hq][D*B*2C][d] workspace (head-major)
   int64_t S;
   int32_t B, Hq, Hkv, d, D, causal;
   float scale;
