@@ -45,7 +45,7 @@ CONFIGS = {
 DEFAULT_CONFIG = "7b_mha"
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
 # the current kernel (profiles/); configurations without a capture report null.
-MEASURED_TRAFFIC = {("7b_mha", "zsa_bwd_wide_kernel"): 809977856 + 495782912}
+MEASURED_TRAFFIC = {("7b_mha", "zsa_bwd_wide_kernel"): 811013888 + 492664576}
 # Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
 CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
 
