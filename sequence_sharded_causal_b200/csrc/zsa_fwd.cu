@@ -13,7 +13,8 @@
 //    stream: two q heads of one kv group (GQA) or two adjacent q tiles (MHA), so a
 //    K/V tile fetched once feeds 2 x 128 rows of MMAs;
 //  * warp roles: 4 softmax warps per slot (one TMEM lane = one query row per thread),
-//    1 TMA producer warp, 1 MMA warp (one thread issues tcgen05.mma);
+//    1 TMA producer warp, 2 MMA warps (one thread each issues tcgen05.mma: one the QK
+//    list, one the PV list);
 //  * S = Q K^T goes to one TMEM buffer (128 x BK fp32) shared by the slots; the softmax
 //    warps of the slot it belongs to copy it to registers and release it at once
 //    (s_free), apply the global-position mask, keep a running max (rescaling O in TMEM
@@ -24,10 +25,10 @@
 //    all 128B-swizzled TMA tiles; TMEM: S | P0 | P1 | O0 | O1 (512 columns at d = 128).
 // The QK MMAs of a unit run in (key tile, slot) order through the S buffer, each one
 // issued as soon as the previous S has been copied out, so the next tile's scores are
-// computed while the softmax still works on the current one.  The MMA thread issues
-// PV_s(n) just before the QK whose S buffer slot s frees next (the softmax of slot s
-// reads S_s(n+1) right after publishing P_s(n)).  The softmax waits for PV_s(n-1)
-// (pv_done) only before it overwrites P_s or rescales O_s, after its exponentials.
+// computed while the softmax still works on the current one.  PV_s(n) is issued as soon
+// as P_s(n) is published (p_full), by the other issuing thread, so neither list waits
+// behind the other.  The softmax waits for PV_s(n-1) (pv_done) only before it
+// overwrites P_s or rescales O_s, after its exponentials.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -188,7 +189,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       for (int k = 0; ok; ++k) {
         // Claim the next unit of the table (dynamic scheduling: the table is grouped
         // by kv head, so CTAs busy at the same time share that head's K/V in L2) and
-        // hand it to the MMA thread and the softmax warps through the ring.
+        // hand it to the MMA threads and the softmax warps through the ring.
         const int slot = k % kUnitRing;
         if (k >= kUnitRing) ok = mbar_wait(&bars.unit_empty[slot], ((k / kUnitRing) - 1) & 1, wctx);
         if (!ok) break;
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
                         &bars.q_full[s], kb * 64, u.head[s], row0);
           ++q_fills[s];
         }
-        // K runs one tile ahead of V: the MMA thread needs K(n+1) (for QK(n+1)) before
+        // K runs one tile ahead of V: the MMA threads need K(n+1) (for QK(n+1)) before
         // V(n) (for PV(n)).
         for (int n = 0; n <= u.nmax && ok; ++n) {
           if (n < u.nmax) {

@@ -20,7 +20,7 @@ struct FwdArgs {
   float scale;
   int* status;
   uint64_t wait_limit_ns;
-  int inject_stall;        // test hook: MMA thread first waits on a barrier nobody arrives at
+  int inject_stall;        // test hook: the MMA threads first wait on a barrier nobody arrives at
 };
 
 struct BwdArgs {
@@ -40,7 +40,7 @@ struct BwdArgs {
   float scale;
   int* status;
   uint64_t wait_limit_ns;
-  int inject_stall;        // test hook: MMA thread first waits on a barrier nobody arrives at
+  int inject_stall;        // test hook: the MMA threads first wait on a barrier nobody arrives at
 };
 
 // Tiling the forward kernel is built for, per head dim.

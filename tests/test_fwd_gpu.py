@@ -104,7 +104,7 @@ def test_fwd_repeatable_and_stream_async(oracle):
 
 
 def test_wait_timeout_reports_status_and_context_survives(oracle):
-    # The stall hook makes the MMA thread wait on a barrier nothing arrives at; with a
+    # The stall hook makes the MMA threads wait on a barrier nothing arrives at; with a
     # 20 ms limit the wait gives up, the kernel drains what it has in flight, releases
     # TMEM and records ZSA_ERR_TIMEOUT; the context stays usable for a normal launch.
     B, S, Hq, Hkv, d, D = 1, 2048, 4, 2, 128, 2
