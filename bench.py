@@ -42,10 +42,12 @@ CONFIGS = {
     "long": dict(B=1, S=131072, Hq=32, Hkv=8, d=128, D=16, seed=4, stress=0.001,
                  desc="long context: B=1 S=131072 Hq=32 Hkv=8 d=128 D=16, 0.1% Q/K rows x8"),
 }
-DEFAULT_CONFIG = "7b_mha"
+# The largest configuration that fits one GPU, and the one at which the throughput
+# targets (S >= 32K) apply.
+DEFAULT_CONFIG = "long"
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
 # the current kernel (profiles/); configurations without a capture report null.
-MEASURED_TRAFFIC = {("7b_mha", "zsa_bwd_wide_kernel"): 811013888 + 492664576}
+MEASURED_TRAFFIC = {}
 # Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
 CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
 
@@ -321,6 +323,16 @@ def run_zsa(args, c, name):
     else:
         dom, dom_tf = "zsa_fwd_kernel", fwd_tf
     traffic = MEASURED_TRAFFIC.get((name, dom))
+    # the two HBM-bound kernels: algorithmic bytes per launch over their event time
+    pairs = B * S * Hq
+    pre_bytes = pairs * (2 * d * 2 + 4 + 4 * d)    # read O, dO; write Delta, zero dQacc
+    dqc_bytes = pairs * d * (4 + 2)                # read fp32 dQacc; write bf16 dQ
+    hbm_kernels = {
+        "bwd_pre": {"bytes": pre_bytes, "gbs": pre_bytes / (kms[1] * 1e-3) / 1e9,
+                    "frac": pre_bytes / (kms[1] * 1e-3) / 1e9 / hbm},
+        "dq_convert": {"bytes": dqc_bytes, "gbs": dqc_bytes / (kms[3] * 1e-3) / 1e9,
+                       "frac": dqc_bytes / (kms[3] * 1e-3) / 1e9 / hbm},
+        "peak_gbs": hbm, "peak_source": f"{peak_src} copy bandwidth"}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -330,6 +342,7 @@ def run_zsa(args, c, name):
                    "l2": f"inputs larger than L2 ({(q.numel() + k.numel() + v.numel() + do.numel()) * 2 / 2**20:.0f} MiB vs 126 MiB), no flush"},
         "pct_of_peak": 100.0 * value / world / peak,
         "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+        "fwd_frac": fwd_tf / peak, "bwd_frac": bwd_tf / peak, "bwd_main_tflops": main_tf,
         "kernel_ms": {"fwd": kms[0], "bwd_pre": kms[1], "bwd_main": kms[2], "dq_convert": kms[3]},
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": dom_tf, "peak": peak,
                      "unit": "TFLOP/s", "frac": dom_tf / peak, "peak_source": f"{peak_src} bf16 burst",
@@ -337,6 +350,7 @@ def run_zsa(args, c, name):
                      "traffic": traffic},
         "e2e": {"value": job_tflops(ff + bf, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
+        "hbm_kernels": hbm_kernels,
         "gpu_launches": 4 * K,
         "clocks": clk,
     }

@@ -95,6 +95,11 @@ typedef struct {
 /*
  * zsa_partition -- the zigzag index map and the balanced causal tile schedule
  * (host only, no GPU needed).
+ * Defined by: "Folding Tensor and Sequence Parallelism" summary, section 2, attention
+ * layer (a zigzag partition balances causal work across shards; chunks r and 2D-1-r
+ * per shard is the reading taken), and the global-position causal mask of "AutoSP"
+ * summary, section 2.A step 4 (which key tiles a query tile sees).  The unit order is
+ * this library's own definition (the pages give none).
  *   perm_host        [S]  or NULL: perm[r*2C + j] = global position of row j of shard r
  *   inv_perm_host    [S]  or NULL: inverse of perm
  *   shard_tiles_host [D]  or NULL: QK^T tile products (block_q x block_k) of shard r,
@@ -114,18 +119,28 @@ ZSA_API int zsa_partition(const zsa_problem* problem, zsa_tiling* tiling, int32_
                   int64_t cap, int64_t* n_work_out);
 
 /* Workspace bytes needed by zsa_attn_fwd (pass = 0) or zsa_attn_bwd (pass = 1).
+ * No passage defines it: the caller owns all device memory, so the library states how
+ * much scratch each pass needs.
  * The workspace must be device memory, 256-byte aligned, not shared between calls in
  * flight.  fwd: status word + the unit table.  bwd: status word + Delta (fp32
  * [D][B][Hq][2C]) + a dQ accumulator (fp32, head-major [Hq][D*B*2C][d]). */
 ZSA_API int zsa_workspace_bytes(const zsa_problem* problem, int pass, size_t* bytes_out);
 
 /* Forward: o (bf16, Q layout) and lse (fp32 [D][B][Hq][2C]).  q, k, v, o, lse and the
- * workspace are device pointers, 16-byte aligned. */
+ * workspace are device pointers, 16-byte aligned.
+ * Defined by: "Folding Tensor and Sequence Parallelism" summary, section 2, attention
+ * layer (each shard's queries run FlashAttention over the all-gathered K/V), with the
+ * causal mask on global positions ("AutoSP" summary, section 2.A step 4) and GQA head
+ * sharing ("Tensor, pipeline e sequence parallelism", 01 Conceito). */
 ZSA_API int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
                  void* o, float* lse, void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /* Backward: dq (Q layout), dk, dv (K layout), all bf16, overwritten (not accumulated).
- * o and lse must come from zsa_attn_fwd on the same inputs. */
+ * o and lse must come from zsa_attn_fwd on the same inputs.
+ * Defined by: the pages describe only the forward; this is the exact gradient of
+ * <dO, O> for the forward above (the reading taken where the pages are silent), with
+ * dK/dV summed over every shard as the reduce-scatter back to the owning shards of the
+ * "Folding Tensor and Sequence Parallelism" attention layer would deliver them. */
 ZSA_API int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
                  const void* o, const float* lse, const void* dout, void* dq, void* dk,
                  void* dv, void* workspace, size_t ws_bytes, void* cuda_stream);
@@ -134,31 +149,37 @@ ZSA_API int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* 
 #define ZSA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
 /* Backward without a workspace argument and without allocating anything.  The pages
- * have no counterpart to this call: it exists for callers that cannot allocate device
- * memory where they call the backward, such as code running while a stream is being
- * captured into a CUDA graph under a no-allocation rule, plugins inside a host
- * runtime that owns and pre-plans all device memory, or C callers without an
- * allocator of their own.  Arguments and results are those of zsa_attn_bwd; the
- * scratch (status word, Delta, fp32 dQ accumulator) is a fixed static device array of
- * ZSA_NOALLOC_SCRATCH_BYTES that every GPU using this call keeps until the process
- * exits.
+ * have no counterpart to this call.  It exists for callers that cannot allocate device
+ * memory where they call the backward: plugins inside a host runtime that owns and
+ * pre-plans all device memory (they may not call cudaMalloc and get no scratch hook),
+ * or C callers without an allocator of their own.  Arguments and results are those of
+ * zsa_attn_bwd; the scratch (status word, Delta, fp32 dQ accumulator) is a fixed static
+ * device array of ZSA_NOALLOC_SCRATCH_BYTES, resident until the process exits on every
+ * GPU on which the library's module is loaded (under CUDA's eager module loading, every
+ * GPU the process has a context on).
  *  - Problems needing more scratch than that (zsa_workspace_bytes(problem, 1) >
  *    ZSA_NOALLOC_SCRATCH_BYTES) return ZSA_ERR_WORKSPACE before anything is enqueued.
- *  - All calls on a device share the array: calls whose GPU work overlaps (other
- *    streams or host threads) race and produce wrong results.  Each call re-zeroes
- *    what must start at zero.
+ *  - All calls on a device share the array and it keeps the last call's contents:
+ *    calls whose GPU work overlaps (other streams or host threads) race and produce
+ *    wrong results.  Each call re-zeroes what must start at zero.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make it before any stream
  *    capture begins.
- *  - Device-side wait timeouts of this call are not reported (its status word lives in
- *    the static array); waits stay bounded. */
+ *  - zsa_set_wait_limit_ns and zsa_debug_inject_stall apply as for zsa_attn_bwd; a
+ *    device-side wait that gives up is reported by zsa_noalloc_status. */
 ZSA_API int zsa_attn_bwd_noalloc(const zsa_problem* problem, const void* q, const void* k,
                                  const void* v, const void* o, const float* lse,
                                  const void* dout, void* dq, void* dk, void* dv,
                                  void* cuda_stream);
 
+/* Synchronises `cuda_stream`, reads and clears the status word of the current device's
+ * zsa_attn_bwd_noalloc scratch: ZSA_OK, or ZSA_ERR_TIMEOUT if a device-side wait of an
+ * earlier zsa_attn_bwd_noalloc call gave up (its outputs are then undefined). */
+ZSA_API int zsa_noalloc_status(void* cuda_stream);
+
 /* Synchronises `cuda_stream`, reads and clears the status word at the start of
- * `workspace`: ZSA_OK, or ZSA_ERR_TIMEOUT if a device-side wait gave up. */
+ * `workspace`: ZSA_OK, or ZSA_ERR_TIMEOUT if a device-side wait gave up.  Failure
+ * detection of this library (bounded waits); the pages define nothing here. */
 ZSA_API int zsa_device_status(void* workspace, void* cuda_stream);
 
 /* Upper bound, in nanoseconds, on any single device-side wait of later launches
@@ -182,7 +203,7 @@ ZSA_API int zsa_debug_inject_stall(int enable);
 enum { ZSA_TRACE_FWD = 0, ZSA_TRACE_BWD_PRE = 1, ZSA_TRACE_BWD_MAIN = 2, ZSA_TRACE_BWD_DQ = 3 };
 ZSA_API int zsa_trace_events(int which, void* begin_event, void* end_event);
 
-/* Static string for a status code. */
+/* Static string for a status code.  Library bookkeeping; no passage defines it. */
 ZSA_API const char* zsa_status_string(int status);
 
 #ifdef __cplusplus

@@ -30,7 +30,8 @@ ZSA_ERR_TIMEOUT = -6
 
 EXPORTED = ("zsa_partition", "zsa_workspace_bytes", "zsa_attn_fwd", "zsa_attn_bwd",
             "zsa_device_status", "zsa_set_wait_limit_ns", "zsa_debug_inject_stall",
-            "zsa_trace_events", "zsa_attn_bwd_noalloc", "zsa_status_string")
+            "zsa_trace_events", "zsa_attn_bwd_noalloc", "zsa_noalloc_status",
+            "zsa_status_string")
 ZSA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 ZSA_TRACE_FWD, ZSA_TRACE_BWD_PRE, ZSA_TRACE_BWD_MAIN, ZSA_TRACE_BWD_DQ = 0, 1, 2, 3
 
@@ -79,6 +80,7 @@ def lib():
         L.zsa_debug_inject_stall.argtypes = [ctypes.c_int]
         L.zsa_trace_events.argtypes = [ctypes.c_int, vp, vp]
         L.zsa_attn_bwd_noalloc.argtypes = [P(zsa_problem)] + [vp] * 10
+        L.zsa_noalloc_status.argtypes = [vp]
         L.zsa_status_string.argtypes = [ctypes.c_int]
         L.zsa_status_string.restype = ctypes.c_char_p
         for name in EXPORTED[:-1]:
@@ -174,12 +176,18 @@ def zsa_attn_bwd(problem, q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes
 def zsa_attn_bwd_noalloc(problem, q, k, v, o, lse, dout, dq, dk, dv, stream=None):
     """zsa_attn_bwd with the library's fixed static scratch instead of a workspace.
 
-    For callers that cannot allocate device memory at the call site; see include/zsa.h
+    For callers that cannot allocate device memory at the call site (a host runtime
+    that owns all device memory, a C caller without an allocator); see include/zsa.h
     for the size limit and the sharing rules.
     """
     _check(lib().zsa_attn_bwd_noalloc(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                       _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                       _stream(stream)), "zsa_attn_bwd_noalloc")
+
+
+def zsa_noalloc_status(stream=None):
+    """Synchronise; status word of the allocation-free backward's scratch (clears it)."""
+    return lib().zsa_noalloc_status(_stream(stream))
 
 
 def zsa_device_status(workspace, stream=None):

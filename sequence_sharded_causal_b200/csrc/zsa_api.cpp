@@ -12,7 +12,9 @@
 #include <map>
 #include <memory>
 #include <mutex>
+#include <set>
 #include <tuple>
+#include <utility>
 
 #include "../../include/zsa.h"
 #include "zsa_kernels.h"
@@ -127,6 +129,23 @@ size_t bwd_workspace(const zsa_problem* p) {
 }  // namespace
 
 namespace zsa {
+int ensure_smem_attr(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return int(e);
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({func, dev})) return int(cudaSuccess);
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return int(e);
+  done.insert({func, dev});
+  return int(cudaSuccess);
+}
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+int inject_stall() { return g_inject_stall.load(); }
+
 TraceEvents trace_events(int which) {
   TraceEvents t{nullptr, nullptr};
   if (which >= 0 && which < 4) {

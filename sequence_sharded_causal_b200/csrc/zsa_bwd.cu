@@ -13,19 +13,29 @@
 // (the single-GPU stand-in for the reduce-scatter back to the owning shards); dQ is
 // summed across key tiles with fp32 reductions into a workspace accumulator.
 //
-// K3 layout (d = 128; d = 64 uses the same code with half-width accumulators):
-//  * one persistent CTA per SM claims key-tile units from a global counter, grouped by
-//    (b, kv head) and longest first within a group; K and V (128 keys) stay in shared
-//    memory for the whole tile;
-//  * q slots are 64-row tiles (a 64-row tile never straddles a zigzag chunk because
-//    C is a multiple of 64) streamed through a 2-stage ring: Q, dO, lse, Delta;
-//  * TMEM: dV | dK (fp32, 128 lanes = keys) | S^T x2 | dP^T | dQ^T (64 cols each);
-//    P^T and dS^T are written back as bf16 over the columns they came from and feed
-//    the dV / dK MMAs as TMEM A operands; dS^T also goes to shared memory (128B
-//    swizzle) as the MN-major B operand of dQ^T = K^T dS^T, whose A operand is the
-//    resident K tile read as an MN-major (transposed) operand;
-//  * warps: 8 compute warps (two groups split each slot's 64 columns), 4 dQ warps
-//    (TMEM -> fp32 reductions into the dQ accumulator), 1 TMA producer, 1 MMA issuer.
+// K3 has two builds, chosen by head dim; both use one persistent CTA per SM that
+// claims key-tile units from a global counter in (b, kv head, key tile) order, keep the
+// unit's K and V tiles (128 keys) in shared memory, stream the q slots that see the tile
+// through a 2-stage TMA ring (Q, dO, lse, Delta), and bound every mbarrier wait.
+//
+//  zsa_bwd_wide_kernel (d <= 128):
+//   * 128-row q slots, so all five MMAs of a slot are N = 128; a 128-row slot may
+//     straddle two zigzag chunks, so the 8 compute warps work in two groups of 64
+//     rows, each over contiguous positions;
+//   * TMEM: dV | dK (fp32, lanes = keys) | ST | XT.  ST receives S^T, then the bf16 P^T
+//     and dS^T (TMEM A operands of dV and dK); XT receives dP^T and, once the compute
+//     warps have read it, dQ^T = K^T dS^T (A = the resident K tile read MN-major, B =
+//     dS^T in shared memory);
+//   * two MMA-issuing threads: one issues S^T and dP^T, the other dV, dK and dQ^T;
+//   * 4 dQ warps read dQ^T out of TMEM and reduce it into the fp32 accumulator.
+//
+//  zsa_bwd_kernel (d = 256):
+//   * dK + dV of a 128-key tile at d = 256 would fill all of TMEM, so each key tile is
+//     two units, one per 128-wide d chunk; both recompute S^T and dP^T;
+//   * 32-row q slots keep K and V (128 KB) plus the Q/dO ring in shared memory;
+//   * TMEM: dV | dK (the chunk) | S^T x2 | dP^T | dQ^T; dS^T also goes to shared memory
+//     (K-major) as the B operand of dQ^T;
+//   * one MMA-issuing thread; 8 compute warps; 4 dQ warps as above.
 #include <cuda_bf16.h>
 
 #include <type_traits>
@@ -1264,11 +1274,9 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
     if constexpr (kWide) return zsa_bwd_wide_kernel<HD>;
     else return zsa_bwd_kernel<HD>;
   }();
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return int(e);
-    attr_set = true;
+  {
+    const int e = ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem);
+    if (e != int(cudaSuccess)) return e;
   }
   const int grid = p.n_units < sms ? p.n_units : sms;
   const TraceEvents tr = trace_events(2);

@@ -555,11 +555,9 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   p.wait_limit_ns = a.wait_limit_ns;
   p.inject_stall = a.inject_stall;
   const int smem = Cfg::SMEM_BYTES + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(zsa_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return int(e);
-    attr_set = true;
+  {
+    const int e = ensure_smem_attr(reinterpret_cast<const void*>(zsa_fwd_kernel<HD>), smem);
+    if (e != int(cudaSuccess)) return e;
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

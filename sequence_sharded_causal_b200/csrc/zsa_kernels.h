@@ -56,6 +56,16 @@ struct TraceEvents {
 };
 TraceEvents trace_events(int which);  // which: 0 fwd, 1 bwd pre, 2 bwd main, 3 dQ convert
 
+// Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once
+// per (kernel, device): cudaFuncSetAttribute applies to the device current at the time
+// of the call only.  Thread-safe.  Returns a cudaError_t.
+int ensure_smem_attr(const void* func, int bytes);
+
+// Wait limit and stall hook set through zsa_set_wait_limit_ns / zsa_debug_inject_stall;
+// every entry point that launches a kernel reads them.
+uint64_t wait_limit_ns();
+int inject_stall();
+
 // Returns a cudaError_t (cudaSuccess on success).
 int launch_fwd(const FwdArgs& a, cudaStream_t stream);
 int launch_bwd(const BwdArgs& a, cudaStream_t stream);

@@ -1,17 +1,18 @@
 // zsa_noalloc.cu -- the backward pass for callers that cannot allocate device memory.
 //
 // zsa_attn_bwd needs a caller-provided workspace (status word, Delta, fp32 dQ
-// accumulator).  Some callers have no way to provide one at the call site: code that
-// runs while a stream is being captured into a CUDA graph under a no-allocation rule,
-// plugins inside a host runtime whose device memory is entirely owned and pre-planned
-// by that runtime, or a C caller that links the library without any allocator of its
-// own.  zsa_attn_bwd_noalloc serves them: its scratch is a file-scope __device__ array
-// of fixed size (ZSA_NOALLOC_SCRATCH_BYTES), so the call itself allocates nothing.
-// The same backward kernels run; only the scratch pointers differ.
+// accumulator).  Some callers have no way to provide one at the call site: plugins
+// inside a host runtime whose device memory is entirely owned and pre-planned by that
+// runtime (they may not call cudaMalloc, and the runtime offers no scratch hook), or a
+// C caller that links the library without any allocator of its own.
+// zsa_attn_bwd_noalloc serves them: its scratch is a file-scope __device__ array of
+// fixed size (ZSA_NOALLOC_SCRATCH_BYTES), so the call itself allocates nothing.  The
+// same backward kernels run; only the scratch pointers differ.
 //
 // Costs and rules, stated for users:
 //  * every GPU on which this library's module is loaded keeps the array resident until
-//    the process exits;
+//    the process exits (with CUDA's eager module loading that is every GPU the process
+//    creates a context on, whether or not it ever calls this entry point);
 //  * problems whose scratch need (the same number zsa_workspace_bytes(problem, 1)
 //    reports) exceeds ZSA_NOALLOC_SCRATCH_BYTES are rejected with ZSA_ERR_WORKSPACE
 //    before anything is enqueued;
@@ -22,9 +23,9 @@
 //  * the first call on each device looks up the array's device address
 //    (cudaGetSymbolAddress) with that device current; make that first call before
 //    any stream capture begins;
-//  * the status word lives in the array, so a device-side wait timeout of this variant
-//    is not reported to the caller (every wait is still bounded; the outputs of such a
-//    call are undefined).
+//  * the wait limit and the stall hook (zsa_set_wait_limit_ns, zsa_debug_inject_stall)
+//    apply as they do to zsa_attn_bwd; a wait that gives up records a timeout in the
+//    status word inside the array, which zsa_noalloc_status reads and clears.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -104,10 +105,25 @@ extern "C" int zsa_attn_bwd_noalloc(const zsa_problem* problem, const void* q, c
   a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
   a.scale = problem->softmax_scale;
   a.status = reinterpret_cast<int*>(base);
-  a.wait_limit_ns = 2000000000ull;
-  a.inject_stall = 0;
+  a.wait_limit_ns = zsa::wait_limit_ns();
+  a.inject_stall = zsa::inject_stall();
   const int e = zsa::launch_bwd(a, stream);
   if (e == int(cudaErrorNotSupported)) return ZSA_ERR_UNSUPPORTED;
   if (e != int(cudaSuccess)) return ZSA_ERR_CUDA;
   return ZSA_OK;
+}
+
+extern "C" int zsa_noalloc_status(void* cuda_stream) {
+  void* scratch = nullptr;
+  int rc = scratch_address(&scratch);
+  if (rc != ZSA_OK) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  int st = 0;
+  if (cudaMemcpyAsync(&st, scratch, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return ZSA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  if (st == 0) return ZSA_OK;
+  if (cudaMemsetAsync(scratch, 0, sizeof(int), stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  return ZSA_ERR_TIMEOUT;
 }

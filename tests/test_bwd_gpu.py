@@ -64,7 +64,9 @@ def test_bwd_matches_oracle(oracle, B, S, Hq, Hkv, d, D, causal, seed):
 
 @pytest.mark.parametrize("B,S,Hq,Hkv,d,D,seed,frac", [
     (1, 2048, 4, 2, 128, 4, 41, 0.01), (1, 1024, 2, 2, 64, 2, 42, 0.02),
-    (1, 1024, 6, 1, 256, 2, 43, 0.02)])
+    (1, 1024, 6, 1, 256, 2, 43, 0.02),
+    (1, 2048, 12, 2, 256, 4, 44, 0.01),    # the wide-head shape's G = 6 and D = 4
+    (1, 4096, 8, 2, 128, 16, 45, 0.01)])   # the long-context G = 4 and D = 16
 def test_bwd_stress_rows(oracle, B, S, Hq, Hkv, d, D, seed, frac):
     q_nat, k, v, do_nat, pos = inputs.make_inputs(B, S, Hq, Hkv, d, seed, stress_frac=frac)
     assert pos.numel() > 0

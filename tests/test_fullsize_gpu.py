@@ -12,7 +12,8 @@ The fp64 oracle cannot run full-size attention, so:
     sum to 0): per kv head, sum_k dV_k = sum of dO over the group's q rows (to 1e-2 of
     that sum), and sum_k dK_k = 0 (to 1e-2 of sum_k |dK_k|, the mass that cancels);
 and, at a reduced sequence length with the same heads, d and D, a full elementwise
-forward + backward check against the full oracle.
+forward + backward check against the full oracle (for the long-context configuration
+with 1% of the Q and K rows scaled x8, so every stressed row is compared elementwise).
 
 Inputs follow the recipe of sequence_sharded_causal_b200.inputs (seeds 1..4 for the
 four configurations).  Tolerances: O max-abs 1e-2 beyond bf16 output rounding, lse
@@ -27,11 +28,13 @@ from sequence_sharded_causal_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
-FULL = {  # name: (B, S, Hq, Hkv, d, D, seed, stress_frac, reduced S)
-    "7b_mha": (1, 16384, 32, 32, 128, 8, 1, 0.0, 4096),
-    "8b_gqa": (1, 32768, 32, 8, 128, 8, 2, 0.0, 4096),
-    "wide_gqa": (1, 65536, 24, 4, 256, 4, 3, 0.0, 2048),
-    "long": (1, 131072, 32, 8, 128, 16, 4, 0.001, None),
+FULL = {  # name: (B, S, Hq, Hkv, d, D, seed, stress_frac, reduced S, reduced-S stress_frac)
+    "7b_mha": (1, 16384, 32, 32, 128, 8, 1, 0.0, 4096, 0.0),
+    "8b_gqa": (1, 32768, 32, 8, 128, 8, 2, 0.0, 4096, 0.0),
+    "wide_gqa": (1, 65536, 24, 4, 256, 4, 3, 0.0, 2048, 0.0),
+    # the long-context heads and shard count (D = 16, C = 128 at S = 4096), with 1% of
+    # the Q and K rows scaled x8 so that about 41 stressed rows land in the reduced case
+    "long": (1, 131072, 32, 8, 128, 16, 4, 0.001, 4096, 0.01),
 }
 O_TOL, LSE_TOL, REL_TOL = 1e-2, 1e-3, 1e-2
 
@@ -64,7 +67,7 @@ def sample_positions(S, D, seed, extra):
 
 @pytest.mark.parametrize("name", list(FULL))
 def test_full_size_sampled_rows(oracle, name):
-    B, S, Hq, Hkv, d, D, seed, frac, _ = FULL[name]
+    B, S, Hq, Hkv, d, D, seed, frac, _, _ = FULL[name]
     q_nat, k, v, do_nat, stress = inputs.make_inputs(B, S, Hq, Hkv, d, seed, stress_frac=frac)
     perm, inv = oracle.partition(S, D)
     q = inputs.to_shard_major(q_nat, perm, D)
@@ -109,8 +112,10 @@ def test_full_size_sampled_rows(oracle, name):
 
 @pytest.mark.parametrize("name", [n for n in FULL if FULL[n][8]])
 def test_reduced_length_full_check(oracle, name):
-    B, _, Hq, Hkv, d, D, seed, _, S = FULL[name]
-    q_nat, k, v, do_nat, _ = inputs.make_inputs(B, S, Hq, Hkv, d, seed + 100)
+    B, _, Hq, Hkv, d, D, seed, _, S, frac = FULL[name]
+    q_nat, k, v, do_nat, stress = inputs.make_inputs(B, S, Hq, Hkv, d, seed + 100,
+                                                     stress_frac=frac)
+    assert (stress.numel() > 0) == (frac > 0)
     perm, _ = oracle.partition(S, D)
     q = inputs.to_shard_major(q_nat, perm, D)
     do = inputs.to_shard_major(do_nat, perm, D)

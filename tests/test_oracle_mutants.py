@@ -70,14 +70,15 @@ def _pins_pass():
     # schedule kend vs brute visibility, and order
     S, D, bq, bk = 512, 2, 64, 64
     perm, _ = oracle.partition(S, D)
-    st, units = oracle.schedule(S, D, 1, 2, 1, True, bq, bk, 2)
+    B_, Hq_, Hkv_ = 1, 2, 1
+    st, units = oracle.schedule(S, D, B_, Hq_, Hkv_, True, bq, bk, 2)
     for u in units:
         r, i0, k0 = int(u[0]), int(u[3]), int(u[7])
         rows = perm[r * (S // D) + i0 * bq: r * (S // D) + (i0 + 1) * bq]
         if k0 != int(rows.max()) // bk + 1:
             return False
     work = np.maximum(units[:, 7], units[:, 8])
-    grp = units[:, 1] * 1 + units[:, 2]
+    grp = units[:, 1] * Hkv_ + units[:, 2]
     if not (np.diff(grp) >= 0).all() or not (np.diff(work)[np.diff(grp) == 0] <= 0).all():
         return False
     # forward vs unsharded brute force (GQA, causal)

@@ -1,12 +1,13 @@
 """The allocation-free backward entry point (zsa_attn_bwd_noalloc).
 
-Some callers cannot allocate device memory where they call the backward (a stream
-being captured under a no-allocation rule, a host runtime that owns all device
-memory): zsa_attn_bwd_noalloc runs the same backward with a fixed static scratch.
-This file checks, through the C ABI, that two calls in a row give the same dQ/dK/dV
-as zsa_attn_bwd with a caller workspace, within the backward's parity tolerance
-(relative Frobenius 1e-2), and that a problem too large for the scratch is refused
-before anything runs.  It is named to be collected last.
+Some callers cannot allocate device memory where they call the backward (a plugin
+inside a host runtime that owns and pre-plans all device memory, a C caller without
+an allocator): zsa_attn_bwd_noalloc runs the same backward with a fixed static
+scratch.  This file checks, through the C ABI, that two calls in a row give the same
+dQ/dK/dV as zsa_attn_bwd with a caller workspace, within the backward's parity
+tolerance (relative Frobenius 1e-2); that a problem too large for the scratch is
+refused before anything runs; and that the wait limit and stall hook reach this entry
+point, with a timeout reported by zsa_noalloc_status.  It is named to be collected last.
 """
 import ctypes
 
@@ -58,3 +59,35 @@ def test_noalloc_matches_workspace_backward_twice():
         for got, want in zip((dq, dk, dv), ref):
             assert torch.isfinite(got.float()).all()
             assert rel_fro(got, want) <= REL_TOL
+
+
+@pytest.mark.gpu
+def test_noalloc_timeout_is_reported_and_next_call_is_clean():
+    # The stall hook makes the MMA threads wait on a barrier nothing arrives at; with a
+    # 20 ms limit that wait gives up, the kernel tears down and records a timeout in the
+    # status word inside the static scratch.  zsa_noalloc_status reports and clears it.
+    B, S, Hq, Hkv, d, D = 1, 1024, 4, 2, 128, 2
+    q_nat, k, v, do_nat, _ = inputs.make_inputs(B, S, Hq, Hkv, d, 52)
+    problem = zsa.make_problem(B, S, Hq, Hkv, d, D)
+    perm = zsa.zsa_partition(problem, want_schedule=False)["perm"]
+    dev = torch.device("cuda", 0)
+    q = inputs.to_shard_major(q_nat, perm, D).to(dev)
+    do = inputs.to_shard_major(do_nat, perm, D).to(dev)
+    k, v = k.to(dev), v.to(dev)
+    o, lse = zsa.attn_fwd(q, k, v, D)
+    ref = zsa.attn_bwd(q, k, v, o, lse, do, D)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    assert zsa.zsa_noalloc_status() == zsa.ZSA_OK
+    try:
+        zsa.zsa_set_wait_limit_ns(20_000_000)
+        zsa.zsa_debug_inject_stall(True)
+        zsa.zsa_attn_bwd_noalloc(problem, q, k, v, o, lse, do, dq, dk, dv)
+        assert zsa.zsa_noalloc_status() == zsa.ZSA_ERR_TIMEOUT
+    finally:
+        zsa.zsa_debug_inject_stall(False)
+        zsa.zsa_set_wait_limit_ns(2_000_000_000)
+    assert zsa.zsa_noalloc_status() == zsa.ZSA_OK        # read-and-clear
+    zsa.zsa_attn_bwd_noalloc(problem, q, k, v, o, lse, do, dq, dk, dv)
+    assert zsa.zsa_noalloc_status() == zsa.ZSA_OK
+    for got, want in zip((dq, dk, dv), ref):
+        assert rel_fro(got, want) <= REL_TOL
