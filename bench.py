@@ -9,8 +9,11 @@ forward (zsa_attn_fwd: zigzag schedule + forward kernel) and the backward
 shards in one launch each.  Throughput is algorithmic causal FLOPs per second:
 forward 4*B*Hq*d*S(S+1)/2, backward 2.5x that.
 
---gpus N > 1 runs N independent replicas (the single-GPU path has no collective;
-launch with torchrun); value is the sum over ranks, time the max over ranks.
+--gpus N > 1 (launched with torchrun, one rank per GPU) runs the D-GPU realisation of the
+same problem: rank q owns D/N of the logical zigzag shards, all-gathers K/V (NCCL) in
+the shard-major order the kernels read, runs the forward and backward over its own
+shards, and reduce-scatters dK/dV back to the owners; value is the whole problem's
+FLOPs over the slowest rank's time (strong scaling).
 --impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
 Prints ONE JSON line on rank 0.
 """
@@ -212,21 +215,48 @@ def run_zsa(args, c, name):
     B, S, Hq, Hkv, d, D = (c[k] for k in ("B", "S", "Hq", "Hkv", "d", "D"))
     problem = zsa.make_problem(B, S, Hq, Hkv, d, D, causal=True)
     perm = zsa.zsa_partition(problem, want_schedule=False)["perm"]
-    q_nat, k, v, do_nat, _ = inputs.make_inputs(B, S, Hq, Hkv, d, c["seed"] + 1000 * rank,
-                                                c["stress"], device=dev)
+    # every rank draws the same problem and keeps its own rows
+    q_nat, k, v, do_nat, _ = inputs.make_inputs(B, S, Hq, Hkv, d, c["seed"], c["stress"],
+                                                device=dev)
     q = inputs.to_shard_major(q_nat, perm, D)
     do = inputs.to_shard_major(do_nat, perm, D)
     del q_nat, do_nat
-    o = torch.empty_like(q)
-    lse = torch.empty(D, B, Hq, S // D, dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws_f = torch.empty(zsa.zsa_workspace_bytes(problem, 0), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(zsa.zsa_workspace_bytes(problem, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if world == 1:
+        # one launch over all D shards, natural-order K/V (the gathered buffer)
+        o = torch.empty_like(q)
+        lse = torch.empty(D, B, Hq, S // D, dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws_f = torch.empty(zsa.zsa_workspace_bytes(problem, 0), dtype=torch.uint8, device=dev)
+        ws_b = torch.empty(zsa.zsa_workspace_bytes(problem, 1), dtype=torch.uint8, device=dev)
 
-    def step():
-        zsa.zsa_attn_fwd(problem, q, k, v, o, lse, ws_f, stream=stream)
-        zsa.zsa_attn_bwd(problem, q, k, v, o, lse, do, dq, dk, dv, ws_b, stream=stream)
+        def step():
+            zsa.zsa_attn_fwd(problem, q, k, v, o, lse, ws_f, stream=stream)
+            zsa.zsa_attn_bwd(problem, q, k, v, o, lse, do, dq, dk, dv, ws_b, stream=stream)
+
+        def device_status():
+            return zsa.zsa_device_status(ws_f) or zsa.zsa_device_status(ws_b)
+        inputs_t, outputs_t = (q, k, v, do), (o, lse, dq, dk, dv)
+    else:
+        from sequence_sharded_causal_b200 import dist as zdist
+        core = zdist.ShardedAttention(B, S, Hq, Hkv, d, D, rank, world, device=dev)
+        s0, ns = core.shard_begin, core.shard_count
+        q = q[s0:s0 + ns].contiguous()
+        do = do[s0:s0 + ns].contiguous()
+        k = inputs.to_shard_major(k, perm, D)[s0:s0 + ns].contiguous()   # the rank's own K/V rows
+        v = inputs.to_shard_major(v, perm, D)[s0:s0 + ns].contiguous()
+        torch.cuda.empty_cache()
+        o, dq = torch.empty_like(q), torch.empty_like(q)
+        dk, dv = torch.empty_like(k), torch.empty_like(v)
+        lse = core.lse
+
+        def step():
+            core.forward(q, k, v, o, stream=stream)
+            core.backward(q, o, do, dq, dk, dv, stream=stream)
+
+        def device_status():
+            return core.status()
+        inputs_t, outputs_t = (q, k, v, do), (o, lse, dq, dk, dv)
 
     def barrier():
         if dist is not None:
@@ -235,7 +265,7 @@ def run_zsa(args, c, name):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    status = zsa.zsa_device_status(ws_f) or zsa.zsa_device_status(ws_b)
+    status = device_status()
     if status != zsa.ZSA_OK:
         raise RuntimeError(f"device status after warm-up: {zsa.status_string(status)}")
 
@@ -270,7 +300,7 @@ def run_zsa(args, c, name):
     barrier()
     for which in range(4):
         zsa.zsa_trace_events(which, None, None)
-    status = zsa.zsa_device_status(ws_f) or zsa.zsa_device_status(ws_b)
+    status = device_status()
     if status != zsa.ZSA_OK:
         raise RuntimeError(f"device status after timing: {zsa.status_string(status)}")
     ms = e0.elapsed_time(e1) / K
@@ -280,10 +310,10 @@ def run_zsa(args, c, name):
 
     # ---- end to end through the API with host buffers (copies inside the timed region)
     pin = dict(pin_memory=True)
-    h_in = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in (q, k, v, do)]
-    for hsrc, dsrc in zip(h_in, (q, k, v, do)):
+    h_in = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in inputs_t]
+    for hsrc, dsrc in zip(h_in, inputs_t):
         hsrc.copy_(dsrc)
-    h_out = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in (o, lse, dq, dk, dv)]
+    h_out = [torch.empty(x.shape, dtype=x.dtype, **pin) for x in outputs_t]
     bi = sum(x.numel() * x.element_size() for x in h_in)
     bo = sum(x.numel() * x.element_size() for x in h_out)
     K2 = max(1, min(K, 10))
@@ -294,10 +324,10 @@ def run_zsa(args, c, name):
     x1 = torch.cuda.Event(enable_timing=True)
     x0.record(stream)
     for _ in range(K2):
-        for dst, src in zip((q, k, v, do), h_in):
+        for dst, src in zip(inputs_t, h_in):
             dst.copy_(src, non_blocking=True)
         step()
-        for dst, src in zip(h_out, (o, lse, dq, dk, dv)):
+        for dst, src in zip(h_out, outputs_t):
             dst.copy_(src, non_blocking=True)
     x1.record(stream)
     torch.cuda.synchronize(dev)
@@ -312,11 +342,13 @@ def run_zsa(args, c, name):
     peak, peak_sus, hbm, peak_src = load_peaks()
     ff = fwd_flops(c)
     bf = 2.5 * ff
-    value = job_tflops(ff + bf, world, ms)
-    fwd_tf = ff / (kms[0] * 1e-3) / 1e12
+    # every rank's share of the problem, summed, over the slowest rank's time
+    value = job_tflops((ff + bf) / world, world, ms)
+    # kernel figures are this rank's: its kernels do 1/world of the problem
+    fwd_tf = ff / world / (kms[0] * 1e-3) / 1e12
     bwd_ms = kms[1] + kms[2] + kms[3]
-    bwd_tf = bf / (bwd_ms * 1e-3) / 1e12
-    main_tf = bf / (kms[2] * 1e-3) / 1e12
+    bwd_tf = bf / world / (bwd_ms * 1e-3) / 1e12
+    main_tf = bf / world / (kms[2] * 1e-3) / 1e12
     # dominant kernel by time: forward kernel or backward main kernel
     if kms[2] >= kms[0]:
         dom, dom_tf = ("zsa_bwd_wide_kernel" if d <= 128 else "zsa_bwd_kernel"), main_tf
@@ -324,7 +356,7 @@ def run_zsa(args, c, name):
         dom, dom_tf = "zsa_fwd_kernel", fwd_tf
     traffic = MEASURED_TRAFFIC.get((name, dom))
     # the two HBM-bound kernels: algorithmic bytes per launch over their event time
-    pairs = B * S * Hq
+    pairs = B * S * Hq // world
     pre_bytes = pairs * (2 * d * 2 + 4 + 4 * d)    # read O, dO; write Delta, zero dQacc
     dqc_bytes = pairs * d * (4 + 2)                # read fp32 dQacc; write bf16 dQ
     hbm_kernels = {
@@ -335,12 +367,16 @@ def run_zsa(args, c, name):
         "peak_gbs": hbm, "peak_source": f"{peak_src} copy bandwidth"}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if world > 1 else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": c["desc"], "B": B, "S": S, "Hq": Hq, "Hkv": Hkv, "d": d, "D": D,
-                   "causal": True, "parallelism": "replicas" if world > 1 else "single",
+                   "causal": True,
+                   "parallelism": f"sp{world}: {D // world} zigzag shards per rank, NCCL "
+                                  "all-gather K/V + reduce-scatter dK/dV" if world > 1 else "single",
                    "l2": f"inputs larger than L2 ({(q.numel() + k.numel() + v.numel() + do.numel()) * 2 / 2**20:.0f} MiB vs 126 MiB), no flush"},
         "pct_of_peak": 100.0 * value / world / peak,
+        "kv_layout": "natural" if world == 1 else "shard-major (all-gather order)",
         "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
         "fwd_frac": fwd_tf / peak, "bwd_frac": bwd_tf / peak, "bwd_main_tflops": main_tf,
         "kernel_ms": {"fwd": kms[0], "bwd_pre": kms[1], "bwd_main": kms[2], "dq_convert": kms[3]},
@@ -348,7 +384,7 @@ def run_zsa(args, c, name):
                      "unit": "TFLOP/s", "frac": dom_tf / peak, "peak_source": f"{peak_src} bf16 burst",
                      "frac_of_sustained": (dom_tf / peak_sus) if peak_sus else None,
                      "traffic": traffic},
-        "e2e": {"value": job_tflops(ff + bf, world, e2e_ms), "unit": "TFLOP/s",
+        "e2e": {"value": job_tflops((ff + bf) / world, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
         "hbm_kernels": hbm_kernels,
         "gpu_launches": 4 * K,

@@ -57,7 +57,8 @@ extern "C" {
 
 enum {
   ZSA_OK = 0,
-  ZSA_ERR_INVALID = -1,     /* null pointer, non-positive size or scale, misaligned pointer  */
+  ZSA_ERR_INVALID = -1,     /* null pointer, non-positive size or scale, misaligned pointer,
+                               bad kv_layout or shard range                                 */
   ZSA_ERR_SHAPE = -2,       /* S % (2*D*64) != 0, Hq % Hkv != 0                              */
   ZSA_ERR_UNSUPPORTED = -3, /* head dim not in {64, 128, 256}; device is not sm_100          */
   ZSA_ERR_WORKSPACE = -4,   /* workspace (or schedule capacity) too small                    */
@@ -65,14 +66,37 @@ enum {
   ZSA_ERR_TIMEOUT = -6      /* a bounded device-side wait gave up (see zsa_device_status)   */
 };
 
-/* One attention problem.  softmax_scale is applied as an fp32 value (callers usually
- * pass 1/sqrt(d) rounded to fp32).  causal = 0 gives full (non-causal) attention with
- * the same layouts. */
+/* K / V layouts (zsa_problem.kv_layout). */
+enum {
+  ZSA_KV_NATURAL = 0,     /* K, V, dK, dV : [B][S][Hkv][d] in position order               */
+  ZSA_KV_SHARD_MAJOR = 1  /* K, V, dK, dV : [D][B][2C][Hkv][d], rows in the Q layout's
+                             zigzag order: exactly what an all-gather of every shard's own
+                             K/V rows produces, and what a reduce-scatter of dK/dV back to
+                             the owning shards consumes, with no reorder pass           */
+};
+
+/* One attention problem, and the part of it one call computes.
+ *  softmax_scale: applied as an fp32 value (callers usually pass 1/sqrt(d) rounded to
+ *    fp32).  causal = 0 gives full (non-causal) attention with the same layouts.
+ *  kv_layout: ZSA_KV_NATURAL or ZSA_KV_SHARD_MAJOR (above); K/V always hold the whole
+ *    gathered sequence.
+ *  shard_begin, shard_count: the call computes the queries of the logical shards
+ *    [shard_begin, shard_begin + shard_count) only (shard_count = 0: all D shards).  The
+ *    Q-layout tensors (Q, O, dO, dQ, lse) then hold just those shards, [shard_count][B]
+ *    [2C][Hq][d] (lse [shard_count][B][Hq][2C]), and dK/dV are the partial sums over
+ *    those shards' queries: one rank's share of a D-rank run, whose reduce-scatter gives
+ *    every owner its slab.  A zero-initialised struct tail keeps the one-launch default
+ *    (natural K/V, all shards).
+ * The sharded reading ("Folding Tensor and Sequence Parallelism" summary, section 2,
+ * attention layer: each rank holds one zigzag shard and an all-gather rebuilds the K/V
+ * context) is what the shard range and the shard-major K/V layout express. */
 typedef struct {
   int64_t B, S;
   int32_t Hq, Hkv, d, D;
   int32_t causal;
   float softmax_scale;
+  int32_t kv_layout;
+  int32_t shard_begin, shard_count;
 } zsa_problem;
 
 /* Tiling of the forward schedule: block_q query rows per tile, block_k keys per key
@@ -145,6 +169,28 @@ ZSA_API int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* 
                  const void* o, const float* lse, const void* dout, void* dq, void* dk,
                  void* dv, void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* Most partial results one zsa_attn_merge call combines. */
+#define ZSA_MERGE_MAX_PARTS 32
+
+/* Merge of partial attention results over disjoint key sets: the combining step of ring
+ * attention ("AutoSP" summary, sections 1 and 4, where ring attention is the
+ * sequence-parallel baseline; the pages give no formula, and the reading taken is the
+ * definition of a softmax over a union of disjoint key sets):
+ *   lse = ln sum_i exp(lse_i),   O = sum_i exp(lse_i - lse) O_i,
+ * an empty key set (lse_i = -inf, O_i = 0) contributing nothing; a (row, head) whose parts
+ * are all empty gets lse = -inf and O = 0.
+ *   problem   : shapes; the Q-layout rows are those of its shard range (all D by default)
+ *   n_parts   : 1 .. ZSA_MERGE_MAX_PARTS
+ *   o_parts   : HOST array of n_parts device pointers, bf16 in the Q layout
+ *   lse_parts : HOST array of n_parts device pointers, fp32 [shards][B][Hq][2C]
+ *   o, lse    : device outputs in the same layouts; they may alias one of the parts (a
+ *               running merge in place)
+ * Pointers 16-byte aligned.  Asynchronous on cuda_stream; HBM-bound (reads n_parts *
+ * (2d + 4) bytes and writes 2d + 4 per (row, head)). */
+ZSA_API int zsa_attn_merge(const zsa_problem* problem, int32_t n_parts, const void* const* o_parts,
+                           const float* const* lse_parts, void* o, float* lse,
+                           void* cuda_stream);
+
 /* Size of the fixed device scratch behind zsa_attn_bwd_noalloc (64 MiB per device). */
 #define ZSA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
@@ -199,8 +245,11 @@ ZSA_API int zsa_debug_inject_stall(int enable);
  * launch stream immediately before / after the kernel, so the caller can time that
  * kernel alone with cudaEventElapsedTime.  which: ZSA_TRACE_FWD (forward kernel),
  * ZSA_TRACE_BWD_PRE (Delta preprocess), ZSA_TRACE_BWD_MAIN (backward main kernel),
- * ZSA_TRACE_BWD_DQ (dQ conversion).  Pass NULL events to stop tracing that kernel. */
-enum { ZSA_TRACE_FWD = 0, ZSA_TRACE_BWD_PRE = 1, ZSA_TRACE_BWD_MAIN = 2, ZSA_TRACE_BWD_DQ = 3 };
+ * ZSA_TRACE_BWD_DQ (dQ conversion), ZSA_TRACE_MERGE (partial-result merge).  Pass NULL events to stop tracing that kernel. */
+enum {
+  ZSA_TRACE_FWD = 0, ZSA_TRACE_BWD_PRE = 1, ZSA_TRACE_BWD_MAIN = 2, ZSA_TRACE_BWD_DQ = 3,
+  ZSA_TRACE_MERGE = 4
+};
 ZSA_API int zsa_trace_events(int which, void* begin_event, void* end_event);
 
 /* Static string for a status code.  Library bookkeeping; no passage defines it. */

@@ -12,6 +12,9 @@ only marshals numpy arrays.  Sources followed:
     recomputed in global positions under sequence sharding.
   * "Tensor, pipeline e sequence parallelism" (llmdeepdive 5.8), "01 Conceito":
     grouped-query heads (q heads share kv heads).
+  * "AutoSP" (gist.science 2604.27089), sections 1 and 4: ring attention, the
+    sequence-parallel baseline whose per-block partial results attn_fwd_keys computes
+    and attn_merge combines (log-sum-exp merge; the reading is stated in oracle.c).
 
 Every function here is pinned by tests/test_oracle_pins.py (brute force, closed
 forms, finite differences, invariants); none is "parity unpinned".
@@ -47,6 +50,11 @@ def _load():
         lib.oracle_attn_dq_rows.argtypes = [i32, i64, i32, i32, i32, i32, i32, dbl, p, i64,
                                             p, p, p, p, p]
         lib.oracle_attn_dq_rows.restype = ctypes.c_int
+        lib.oracle_attn_fwd_keys.argtypes = [i32, i64, i32, i32, i32, i32, i32, dbl, i64, i64,
+                                             p, p, p, p, p]
+        lib.oracle_attn_fwd_keys.restype = ctypes.c_int
+        lib.oracle_attn_merge.argtypes = [i32, i64, i32, p, p, p, p]
+        lib.oracle_attn_merge.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -180,3 +188,45 @@ def attn_bwd(q, k, v, dout, D, causal=True, scale=None):
     if rc != 0:
         raise ValueError("oracle_attn_bwd: invalid problem")
     return dict(dq=dq, dk=dk, dv=dv, o=o, lse=lse, delta=delta)
+
+
+def attn_fwd_keys(q, k, v, D, key_lo, key_hi, causal=True, scale=None):
+    """Forward restricted to the keys at positions [key_lo, key_hi) (and k <= p when
+    causal).  Layouts as attn_fwd; rows seeing no key get lse = -inf, O = 0."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    Dq, B, twoC, Hq, d = q.shape
+    Bk, S, Hkv, dk = k.shape
+    assert Dq == D and Bk == B and dk == d and S == D * twoC and v.shape == k.shape
+    if scale is None:
+        scale = float(np.float32(1.0 / np.sqrt(d)))
+    o = np.empty_like(q)
+    lse = np.empty((D, B, Hq, twoC), np.float64)
+    rc = _load().oracle_attn_fwd_keys(B, S, Hq, Hkv, d, D, int(bool(causal)), float(scale),
+                                      int(key_lo), int(key_hi), _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attn_fwd_keys: invalid problem or key range")
+    return o, lse
+
+
+def attn_merge(o_parts, lse_parts):
+    """Merge partial results over disjoint key sets.
+
+    o_parts: list of Q-layout arrays [D'][B][2C][Hq][d]; lse_parts: matching lists of
+    [D'][B][Hq][2C].  Returns (o, lse) in the same layouts, float64.
+    """
+    o_parts = [_f64(x) for x in o_parts]
+    lse_parts = [_f64(x) for x in lse_parts]
+    n = len(o_parts)
+    Dq, B, twoC, Hq, d = o_parts[0].shape
+    m = Dq * B * twoC * Hq
+    # lse [D'][B][Hq][2C] -> the O layout's pair order [D'][B][2C][Hq]
+    lse_pairs = np.ascontiguousarray(np.stack([x.transpose(0, 1, 3, 2) for x in lse_parts]))
+    o_stack = np.ascontiguousarray(np.stack(o_parts))
+    o = np.empty((Dq, B, twoC, Hq, d), np.float64)
+    lse_flat = np.empty((Dq, B, twoC, Hq), np.float64)
+    rc = _load().oracle_attn_merge(n, m, d, _ptr(o_stack), _ptr(lse_pairs), _ptr(o),
+                                   _ptr(lse_flat))
+    if rc != 0:
+        raise ValueError("oracle_attn_merge: invalid arguments")
+    return o, np.ascontiguousarray(lse_flat.transpose(0, 1, 3, 2))

@@ -60,3 +60,34 @@ def causal_attention_bwd(q, k, v, do, causal=True, scale=None):
             dk[b, :, kv, :] += scale * ds.T @ q[b, :, h, :]
             dv[b, :, kv, :] += p.T @ do[b, :, h, :]
     return dq, dk, dv
+
+
+def key_range_attention(q, k, v, key_lo, key_hi, causal=True, scale=None):
+    """Attention restricted to the keys at positions [key_lo, key_hi) (natural order),
+    full-matrix: keys outside the range (or above the diagonal when causal) are masked to
+    -inf; a row with every key masked gets lse = -inf and O = 0.
+    Returns (o [B][S][Hq][d], lse [B][Hq][S])."""
+    q, k, v = (np.asarray(x, np.float64) for x in (q, k, v))
+    B, S, Hq, d = q.shape
+    G = Hq // k.shape[2]
+    if scale is None:
+        scale = float(np.float32(1.0 / np.sqrt(d)))
+    pos = np.arange(S)
+    visible = (pos[None, :] >= key_lo) & (pos[None, :] < key_hi)
+    if causal:
+        visible = visible & (pos[None, :] <= pos[:, None])
+    else:
+        visible = np.broadcast_to(visible, (S, S))
+    o = np.zeros_like(q)
+    lse = np.full((B, Hq, S), -np.inf)
+    rows = visible.any(axis=1)
+    for b in range(B):
+        for h in range(Hq):
+            s = scale * q[b, :, h, :] @ k[b, :, h // G, :].T
+            s = np.where(visible, s, -np.inf)[rows]
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            o[b, rows, h, :] = (e / l) @ v[b, :, h // G, :]
+            lse[b, h, rows] = (m + np.log(l))[:, 0]
+    return o, lse

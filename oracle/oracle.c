@@ -407,3 +407,105 @@ int oracle_attn_dq_rows(int32_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t d
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Partial results over a key range, and their merge                   */
+/* ------------------------------------------------------------------ */
+/*
+ * Ring attention ("AutoSP" summary page, sections 1 and 4, where it is the
+ * sequence-parallel baseline) hands each rank's queries the K/V blocks one after
+ * another; each block gives the softmax attention restricted to its keys, and the
+ * pieces are combined.  The pages print no formula.  The reading taken is the
+ * definition of a softmax over a union of disjoint key sets K_1, ..., K_n: with
+ * lse_i = ln sum_{k in K_i} exp(s_k) and O_i = sum_{k in K_i} exp(s_k - lse_i) v_k,
+ *   lse = ln sum_i exp(lse_i),   O = sum_i exp(lse_i - lse) O_i,
+ * an empty K_i contributing lse_i = -inf and O_i = 0.
+ */
+
+/* Forward restricted to the keys at positions [key_lo, key_hi), intersected with the
+ * causal set k <= p.  A row that sees no key gets lse = -inf and O = 0.
+ * Layouts as oracle_attn_fwd. */
+int oracle_attn_fwd_keys(int32_t B, int64_t S, int32_t Hq, int32_t Hkv, int32_t d,
+                         int32_t D, int32_t causal, double scale, int64_t key_lo,
+                         int64_t key_hi, const double *q, const double *k,
+                         const double *v, double *o, double *lse)
+{
+    if (check_problem(B, S, Hq, Hkv, d, D)) return -1;
+    if (key_lo < 0 || key_hi > S || key_lo > key_hi) return -1;
+    int64_t twoC = S / D;
+    int32_t G = Hq / Hkv;
+    int64_t n_rows = (int64_t)D * B * twoC;
+#pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)S);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t idx = 0; idx < n_rows * Hq; ++idx) {
+            int64_t row = idx / Hq;
+            int32_t h = (int32_t)(idx % Hq);
+            int32_t r = (int32_t)(row / ((int64_t)B * twoC));
+            int32_t b = (int32_t)((row / twoC) % B);
+            int64_t j = row % twoC;
+            int64_t p = zigzag_position(S, D, r, j);
+            int32_t kv = h / G;
+            const double *q_row = q + (row * Hq + h) * d;
+            double *o_row = o + (row * Hq + h) * d;
+            int64_t end = key_hi;
+            if (causal && p + 1 < end) end = p + 1;          /* visible: key <= p */
+            for (int32_t t = 0; t < d; ++t) o_row[t] = 0.0;
+            double *lse_out = &lse[(((int64_t)r * B + b) * Hq + h) * twoC + j];
+            if (end <= key_lo) {                              /* no visible key */
+                *lse_out = -INFINITY;
+                continue;
+            }
+            double m = -INFINITY;
+            for (int64_t key = key_lo; key < end; ++key) {
+                const double *kk = k + (((int64_t)b * S + key) * Hkv + kv) * d;
+                double dot = 0.0;
+                for (int32_t t = 0; t < d; ++t) dot += q_row[t] * kk[t];
+                s_buf[key] = scale * dot;
+                if (s_buf[key] > m) m = s_buf[key];
+            }
+            double l = 0.0;
+            for (int64_t key = key_lo; key < end; ++key) l += exp(s_buf[key] - m);
+            double lse_r = m + log(l);
+            for (int64_t key = key_lo; key < end; ++key) {
+                double pk = exp(s_buf[key] - lse_r);
+                const double *vv = v + (((int64_t)b * S + key) * Hkv + kv) * d;
+                for (int32_t t = 0; t < d; ++t) o_row[t] += pk * vv[t];
+            }
+            *lse_out = lse_r;
+        }
+        free(s_buf);
+    }
+    return 0;
+}
+
+/* Merge of n partial results.  o_parts [n][m][d] and lse_parts [n][m] hold, for the
+ * same m (row, head) pairs in the same order, each part's O and lse; writes o [m][d]
+ * and lse [m].  Pairs whose parts are all empty get lse = -inf and O = 0. */
+int oracle_attn_merge(int32_t n, int64_t m, int32_t d, const double *o_parts,
+                      const double *lse_parts, double *o, double *lse)
+{
+    if (n <= 0 || m < 0 || d <= 0) return -1;
+    for (int64_t x = 0; x < m; ++x) {
+        double mx = -INFINITY;
+        for (int32_t i = 0; i < n; ++i)
+            if (lse_parts[(int64_t)i * m + x] > mx) mx = lse_parts[(int64_t)i * m + x];
+        double *o_row = o + x * d;
+        for (int32_t t = 0; t < d; ++t) o_row[t] = 0.0;
+        if (mx == -INFINITY) {
+            lse[x] = -INFINITY;
+            continue;
+        }
+        double l = 0.0;
+        for (int32_t i = 0; i < n; ++i) l += exp(lse_parts[(int64_t)i * m + x] - mx);
+        double lse_x = mx + log(l);
+        for (int32_t i = 0; i < n; ++i) {
+            double w = exp(lse_parts[(int64_t)i * m + x] - lse_x);
+            const double *oi = o_parts + ((int64_t)i * m + x) * d;
+            for (int32_t t = 0; t < d; ++t) o_row[t] += w * oi[t];
+        }
+        lse[x] = lse_x;
+    }
+    return 0;
+}

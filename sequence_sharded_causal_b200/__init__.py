@@ -9,7 +9,10 @@ attn_fwd / attn_bwd are conveniences that allocate outputs and the workspace thr
 PyTorch (device memory only) and then call the same entry points.
 
 Layouts (see include/zsa.h): Q, O, dO, dQ are shard-major [D][B][2C][Hq][d]; K, V, dK,
-dV are natural-order [B][S][Hkv][d]; lse is fp32 [D][B][Hq][2C]; tensors are bf16.
+dV are natural-order [B][S][Hkv][d] (kv_layout=ZSA_KV_NATURAL) or shard-major
+[D][B][2C][Hkv][d] (ZSA_KV_SHARD_MAJOR); lse is fp32 [D][B][Hq][2C]; tensors are bf16.
+A call restricted to the shards [shard_begin, shard_begin + shard_count) takes the
+Q-layout tensors of those shards only.
 """
 import ctypes
 import math
@@ -27,19 +30,24 @@ ZSA_ERR_UNSUPPORTED = -3
 ZSA_ERR_WORKSPACE = -4
 ZSA_ERR_CUDA = -5
 ZSA_ERR_TIMEOUT = -6
+ZSA_KV_NATURAL = 0
+ZSA_KV_SHARD_MAJOR = 1
 
 EXPORTED = ("zsa_partition", "zsa_workspace_bytes", "zsa_attn_fwd", "zsa_attn_bwd",
             "zsa_device_status", "zsa_set_wait_limit_ns", "zsa_debug_inject_stall",
-            "zsa_trace_events", "zsa_attn_bwd_noalloc", "zsa_noalloc_status",
-            "zsa_status_string")
+            "zsa_trace_events", "zsa_attn_merge", "zsa_attn_bwd_noalloc",
+            "zsa_noalloc_status", "zsa_status_string")
 ZSA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
-ZSA_TRACE_FWD, ZSA_TRACE_BWD_PRE, ZSA_TRACE_BWD_MAIN, ZSA_TRACE_BWD_DQ = 0, 1, 2, 3
+ZSA_TRACE_FWD, ZSA_TRACE_BWD_PRE, ZSA_TRACE_BWD_MAIN, ZSA_TRACE_BWD_DQ, ZSA_TRACE_MERGE = range(5)
+ZSA_MERGE_MAX_PARTS = 32
 
 
 class zsa_problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("S", ctypes.c_int64), ("Hq", ctypes.c_int32),
                 ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("D", ctypes.c_int32),
-                ("causal", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+                ("causal", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("kv_layout", ctypes.c_int32), ("shard_begin", ctypes.c_int32),
+                ("shard_count", ctypes.c_int32)]
 
 
 class zsa_tiling(ctypes.Structure):
@@ -79,6 +87,7 @@ def lib():
         L.zsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.zsa_debug_inject_stall.argtypes = [ctypes.c_int]
         L.zsa_trace_events.argtypes = [ctypes.c_int, vp, vp]
+        L.zsa_attn_merge.argtypes = [P(zsa_problem), ctypes.c_int32, vp, vp, vp, vp, vp]
         L.zsa_attn_bwd_noalloc.argtypes = [P(zsa_problem)] + [vp] * 10
         L.zsa_noalloc_status.argtypes = [vp]
         L.zsa_status_string.argtypes = [ctypes.c_int]
@@ -98,11 +107,13 @@ def _check(rc, where):
         raise ZsaError(rc, where)
 
 
-def make_problem(B, S, Hq, Hkv, d, D, causal=True, scale=None):
+def make_problem(B, S, Hq, Hkv, d, D, causal=True, scale=None, kv_layout=ZSA_KV_NATURAL,
+                 shard_begin=0, shard_count=0):
+    """zsa_problem; shard_count = 0 means all D shards (one launch)."""
     if scale is None:
         scale = float(np.float32(1.0 / math.sqrt(d)))
     return zsa_problem(int(B), int(S), int(Hq), int(Hkv), int(d), int(D), int(bool(causal)),
-                       float(scale))
+                       float(scale), int(kv_layout), int(shard_begin), int(shard_count))
 
 
 def _ptr(x):
@@ -173,6 +184,19 @@ def zsa_attn_bwd(problem, q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes
                               _ptr(workspace), int(ws_bytes), _stream(stream)), "zsa_attn_bwd")
 
 
+def zsa_attn_merge(problem, o_parts, lse_parts, o, lse, stream=None):
+    """Merge partial results (O_i bf16 Q layout, lse_i fp32) over disjoint key sets into
+    o / lse (which may alias a part)."""
+    n = len(o_parts)
+    if n != len(lse_parts):
+        raise ValueError("o_parts and lse_parts differ in length")
+    op = (ctypes.c_void_p * n)(*[_ptr(x) for x in o_parts])
+    lp = (ctypes.c_void_p * n)(*[_ptr(x) for x in lse_parts])
+    _check(lib().zsa_attn_merge(ctypes.byref(problem), n, ctypes.cast(op, ctypes.c_void_p),
+                                ctypes.cast(lp, ctypes.c_void_p), _ptr(o), _ptr(lse),
+                                _stream(stream)), "zsa_attn_merge")
+
+
 def zsa_attn_bwd_noalloc(problem, q, k, v, o, lse, dout, dq, dk, dv, stream=None):
     """zsa_attn_bwd with the library's fixed static scratch instead of a workspace.
 
@@ -231,17 +255,29 @@ def _check_tensor(x, shape, dtype, name):
 
 
 def _shapes(problem):
+    """(Q-layout shape, K/V shape, lse shape) of a problem."""
     B, S, Hq, Hkv, d, D = (int(problem.B), int(problem.S), int(problem.Hq), int(problem.Hkv),
                            int(problem.d), int(problem.D))
-    return (D, B, S // D, Hq, d), (B, S, Hkv, d), (D, B, Hq, S // D)
+    ns = int(problem.shard_count) or D
+    kv = (B, S, Hkv, d) if problem.kv_layout == ZSA_KV_NATURAL else (D, B, S // D, Hkv, d)
+    return (ns, B, S // D, Hq, d), kv, (ns, B, Hq, S // D)
 
 
-def attn_fwd(q, k, v, D, causal=True, scale=None, workspace=None):
-    """O, lse = attention(Q, K, V) with all D zigzag shards in one launch."""
+def _problem_from(q, k, D, causal, scale, kv_layout, shard_begin, shard_count):
+    ns, B, twoC, Hq, d = q.shape
+    S = D * twoC
+    Hkv = k.shape[2] if kv_layout == ZSA_KV_NATURAL else k.shape[3]
+    if shard_count == 0 and ns != D:
+        raise ValueError(f"q holds {ns} shards; pass shard_begin / shard_count for a subset of D={D}")
+    return make_problem(B, S, Hq, Hkv, d, D, causal, scale, kv_layout, shard_begin, shard_count)
+
+
+def attn_fwd(q, k, v, D, causal=True, scale=None, workspace=None, kv_layout=ZSA_KV_NATURAL,
+             shard_begin=0, shard_count=0):
+    """O, lse = attention(Q, K, V): all D zigzag shards in one launch, or the shards
+    [shard_begin, shard_begin + shard_count) when shard_count > 0."""
     import torch
-    Dq, B, twoC, Hq, d = q.shape
-    S = Dq * twoC
-    problem = make_problem(B, S, Hq, k.shape[2], d, D, causal, scale)
+    problem = _problem_from(q, k, D, causal, scale, kv_layout, shard_begin, shard_count)
     qs, ks, ls = _shapes(problem)
     _check_tensor(q, qs, torch.bfloat16, "q")
     _check_tensor(k, ks, torch.bfloat16, "k")
@@ -255,12 +291,12 @@ def attn_fwd(q, k, v, D, causal=True, scale=None, workspace=None):
     return o, lse
 
 
-def attn_bwd(q, k, v, o, lse, do, D, causal=True, scale=None, workspace=None):
-    """dQ, dK, dV of <dO, O> (dK/dV summed over all shards and the q heads of a group)."""
+def attn_bwd(q, k, v, o, lse, do, D, causal=True, scale=None, workspace=None,
+             kv_layout=ZSA_KV_NATURAL, shard_begin=0, shard_count=0):
+    """dQ, dK, dV of <dO, O>: dK/dV summed over the launch's shards (all D by default)
+    and the q heads of a group."""
     import torch
-    Dq, B, twoC, Hq, d = q.shape
-    S = Dq * twoC
-    problem = make_problem(B, S, Hq, k.shape[2], d, D, causal, scale)
+    problem = _problem_from(q, k, D, causal, scale, kv_layout, shard_begin, shard_count)
     qs, ks, ls = _shapes(problem)
     for name, x, shp in (("q", q, qs), ("k", k, ks), ("v", v, ks), ("o", o, qs), ("do", do, qs)):
         _check_tensor(x, shp, torch.bfloat16, name)

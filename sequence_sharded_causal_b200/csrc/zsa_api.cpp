@@ -27,8 +27,9 @@ using zsa::Schedule;
 constexpr size_t kStatusBytes = 256;
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_inject_stall{0};
-std::atomic<void*> g_trace_begin[4];
-std::atomic<void*> g_trace_end[4];
+constexpr int kTraceKernels = 5;
+std::atomic<void*> g_trace_begin[kTraceKernels];
+std::atomic<void*> g_trace_end[kTraceKernels];
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -38,6 +39,11 @@ int check_problem(const zsa_problem* p) {
     return ZSA_ERR_INVALID;
   if (!(p->softmax_scale > 0.0f) || !std::isfinite(p->softmax_scale)) return ZSA_ERR_INVALID;
   if (p->causal != 0 && p->causal != 1) return ZSA_ERR_INVALID;
+  if (p->kv_layout != ZSA_KV_NATURAL && p->kv_layout != ZSA_KV_SHARD_MAJOR) return ZSA_ERR_INVALID;
+  if (p->shard_begin < 0 || p->shard_count < 0 || p->shard_begin >= p->D ||
+      p->shard_begin + (p->shard_count ? p->shard_count : p->D) > p->D)
+    return ZSA_ERR_INVALID;
+  if (p->shard_count == 0 && p->shard_begin != 0) return ZSA_ERR_INVALID;
   if (p->Hq % p->Hkv != 0) return ZSA_ERR_SHAPE;
   if (p->S % (2 * int64_t(p->D) * 64) != 0) return ZSA_ERR_SHAPE;
   if (p->B * p->S >= (int64_t(1) << 31)) return ZSA_ERR_SHAPE;  // TMA row coordinates are int32
@@ -55,6 +61,10 @@ int check_device_problem(const zsa_problem* p) {
 }
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
+
+// Shards a call computes, and its Q-layout rows (shards * B * 2C).
+int32_t local_shards(const zsa_problem* p) { return p->shard_count ? p->shard_count : p->D; }
+int64_t local_rows(const zsa_problem* p) { return int64_t(local_shards(p)) * p->B * (p->S / p->D); }
 
 int check_sm100() {
   static std::mutex mu;
@@ -82,21 +92,25 @@ struct CachedSchedule {
   }
 };
 
-using SchedKey = std::tuple<int64_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t>;
+using SchedKey = std::tuple<int64_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t, int32_t,
+                           int32_t, int32_t, int32_t>;
 
 std::shared_ptr<CachedSchedule> get_schedule(int64_t S, int32_t D, int32_t B, int32_t Hq,
                                              int32_t Hkv, int32_t causal, int32_t bq, int32_t bk,
-                                             int32_t slots, bool want_pinned) {
+                                             int32_t slots, int32_t shard_begin,
+                                             int32_t shard_count, bool want_pinned) {
   static std::mutex mu;
   static std::map<SchedKey, std::shared_ptr<CachedSchedule>> cache;
-  SchedKey key{S, D, B, Hq, Hkv, causal, bq, bk, slots};
+  SchedKey key{S, D, B, Hq, Hkv, causal, bq, bk, slots, shard_begin, shard_count};
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
     if (it != cache.end() && (!want_pinned || it->second->pinned)) return it->second;
   }
   auto e = std::make_shared<CachedSchedule>();
-  if (!zsa::build_schedule(S, D, B, Hq, Hkv, causal, bq, bk, slots, &e->sched)) return nullptr;
+  if (!zsa::build_schedule(S, D, B, Hq, Hkv, causal, bq, bk, slots, shard_begin, shard_count,
+                           &e->sched))
+    return nullptr;
   if (want_pinned) {
     const size_t bytes = e->sched.units.size() * sizeof(zsa::DevUnit);
     void* h = nullptr;
@@ -116,13 +130,13 @@ size_t fwd_workspace(const zsa_problem* p) {
   const int64_t T = (p->S / p->D) / bq;
   const int64_t G = p->Hq / p->Hkv;
   const int64_t runs = (T * G + slots - 1) / slots;
-  const int64_t units = p->B * p->Hkv * p->D * runs;
+  const int64_t units = p->B * p->Hkv * local_shards(p) * runs;
   return kStatusBytes + align256(size_t(units) * sizeof(zsa::DevUnit));
 }
 
 size_t bwd_workspace(const zsa_problem* p) {
-  const size_t stats = size_t(p->B) * p->S * p->Hq * sizeof(float);       // Delta
-  const size_t dqacc = size_t(p->B) * p->S * p->Hq * p->d * sizeof(float);
+  const size_t stats = size_t(local_rows(p)) * p->Hq * sizeof(float);       // Delta
+  const size_t dqacc = size_t(local_rows(p)) * p->Hq * p->d * sizeof(float);
   return kStatusBytes + align256(stats) + align256(dqacc);
 }
 
@@ -148,7 +162,7 @@ int inject_stall() { return g_inject_stall.load(); }
 
 TraceEvents trace_events(int which) {
   TraceEvents t{nullptr, nullptr};
-  if (which >= 0 && which < 4) {
+  if (which >= 0 && which < kTraceKernels) {
     t.begin = static_cast<cudaEvent_t>(g_trace_begin[which].load());
     t.end = static_cast<cudaEvent_t>(g_trace_end[which].load());
   }
@@ -159,7 +173,7 @@ TraceEvents trace_events(int which) {
 extern "C" {
 
 int zsa_trace_events(int which, void* begin_event, void* end_event) {
-  if (which < 0 || which >= 4) return ZSA_ERR_INVALID;
+  if (which < 0 || which >= kTraceKernels) return ZSA_ERR_INVALID;
   g_trace_begin[which].store(begin_event);
   g_trace_end[which].store(end_event);
   return ZSA_OK;
@@ -221,7 +235,7 @@ int zsa_partition(const zsa_problem* problem, zsa_tiling* tiling, int32_t* perm_
   }
   if (!shard_tiles_host && !sched_host && !n_work_out) return ZSA_OK;
   auto cs = get_schedule(S, D, int32_t(problem->B), problem->Hq, problem->Hkv, problem->causal, bq,
-                         bk, slots, false);
+                         bk, slots, problem->shard_begin, local_shards(problem), false);
   if (!cs) return ZSA_ERR_SHAPE;
   const Schedule& sc = cs->sched;
   if (shard_tiles_host)
@@ -264,7 +278,8 @@ int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const
   int32_t bq, bk, slots;
   zsa::fwd_tiling(problem->d, &bq, &bk, &slots);
   auto cs = get_schedule(problem->S, problem->D, int32_t(problem->B), problem->Hq, problem->Hkv,
-                         problem->causal, bq, bk, slots, true);
+                         problem->causal, bq, bk, slots, problem->shard_begin,
+                         local_shards(problem), true);
   if (!cs) return ZSA_ERR_CUDA;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -281,6 +296,9 @@ int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const
   a.S = problem->S; a.B = int32_t(problem->B); a.Hq = problem->Hq; a.Hkv = problem->Hkv;
   a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
   a.scale = problem->softmax_scale;
+  a.kv_layout = problem->kv_layout;
+  a.shard_begin = problem->shard_begin;
+  a.shard_count = local_shards(problem);
   a.status = reinterpret_cast<int*>(ws);
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.inject_stall = g_inject_stall.load();
@@ -304,7 +322,7 @@ int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const
   if (rc) return rc;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t stats = size_t(problem->B) * problem->S * problem->Hq * sizeof(float);
+  const size_t stats = size_t(local_rows(problem)) * problem->Hq * sizeof(float);
   if (cudaMemsetAsync(ws, 0, kStatusBytes, stream) != cudaSuccess) return ZSA_ERR_CUDA;
   zsa::BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
@@ -314,12 +332,41 @@ int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const
   a.S = problem->S; a.B = int32_t(problem->B); a.Hq = problem->Hq; a.Hkv = problem->Hkv;
   a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
   a.scale = problem->softmax_scale;
+  a.kv_layout = problem->kv_layout;
+  a.shard_begin = problem->shard_begin;
+  a.shard_count = local_shards(problem);
   a.status = reinterpret_cast<int*>(ws);
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.inject_stall = g_inject_stall.load();
   const int e = zsa::launch_bwd(a, stream);
   if (e == int(cudaErrorNotSupported)) return ZSA_ERR_UNSUPPORTED;
   if (e != int(cudaSuccess)) return ZSA_ERR_CUDA;
+  return ZSA_OK;
+}
+
+int zsa_attn_merge(const zsa_problem* problem, int32_t n_parts, const void* const* o_parts,
+                   const float* const* lse_parts, void* o, float* lse, void* cuda_stream) {
+  int rc = check_device_problem(problem);
+  if (rc) return rc;
+  if (n_parts < 1 || n_parts > ZSA_MERGE_MAX_PARTS || !o_parts || !lse_parts || !o || !lse)
+    return ZSA_ERR_INVALID;
+  zsa::MergeArgs a;
+  for (int i = 0; i < n_parts; ++i) {
+    if (!o_parts[i] || !lse_parts[i] || !aligned16(o_parts[i]) || !aligned16(lse_parts[i]))
+      return ZSA_ERR_INVALID;
+    a.o[i] = o_parts[i];
+    a.lse[i] = lse_parts[i];
+  }
+  if (!aligned16(o) || !aligned16(lse)) return ZSA_ERR_INVALID;
+  rc = check_sm100();
+  if (rc) return rc;
+  a.o_out = o;
+  a.lse_out = lse;
+  a.S = problem->S;
+  a.rows = local_rows(problem);
+  a.Hq = problem->Hq; a.d = problem->d; a.D = problem->D; a.n = n_parts;
+  if (zsa::launch_merge(a, static_cast<cudaStream_t>(cuda_stream)) != int(cudaSuccess))
+    return ZSA_ERR_CUDA;
   return ZSA_OK;
 }
 

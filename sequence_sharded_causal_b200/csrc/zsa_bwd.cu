@@ -170,6 +170,9 @@ struct BwdParams {
   int32_t n_units, n_qtiles;  // n_qtiles = BQ-row tiles per shard
   int32_t n_chunks, bq;       // d chunks per key tile, query rows per slot
   int32_t n_ktiles;           // S / 128
+  int32_t kv_shard_major;     // K/V/dK/dV rows in the shard-major zigzag order
+  int32_t shard_begin, shard_end;   // the launch computes the queries of these shards
+  int64_t rows;               // local Q-layout rows: (shard_end - shard_begin) * B * 2C
   float scale, scale_log2;
   int* status;
   int* counter;       // next unclaimed unit (zeroed before every launch)
@@ -230,9 +233,10 @@ __device__ __forceinline__ bool tile_sees(const BwdParams& p, int32_t r, int32_t
   return !p.causal || (zz_pos(p.C, p.D, r, int64_t(i) * p.bq + p.bq - 1) >= int64_t(n) * 128);
 }
 
-// First slot at or after (r, i, 0); false when the walk is over.
+// First slot at or after (r, i, 0); false when the walk is over.  Only the launch's
+// shards [shard_begin, shard_end) are walked.
 __device__ __forceinline__ bool walk_seek(const BwdParams& p, int32_t n, SlotWalk& w) {
-  while (w.r < p.D) {
+  while (w.r < p.shard_end) {
     if (tile_sees(p, w.r, w.i, n, &w.p0)) return true;
     if (++w.i == p.n_qtiles) {
       w.i = 0;
@@ -242,7 +246,7 @@ __device__ __forceinline__ bool walk_seek(const BwdParams& p, int32_t n, SlotWal
   return false;
 }
 __device__ __forceinline__ bool walk_first(const BwdParams& p, int32_t n, SlotWalk& w) {
-  w.r = 0; w.i = 0; w.e = 0;
+  w.r = p.shard_begin; w.i = 0; w.e = 0;
   return walk_seek(p, n, w);
 }
 __device__ __forceinline__ bool walk_next(const BwdParams& p, int32_t n, SlotWalk& w) {
@@ -342,10 +346,15 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
         if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
-        const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(u.n) * BKV);
-        for (int kb = 0; kb < KB; ++kb) {
-          tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128, &map_k, &bars.kv_full, kb * 64, u.g, key0);
-          tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128, &map_v, &bars.kv_full, kb * 64, u.g, key0);
+        for (int hb = 0; hb < BKV / 64; ++hb) {
+          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * 64, u.b, prm.S, prm.B, prm.D,
+                                             prm.kv_shard_major);
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128 + hb * 64 * 128, &map_k, &bars.kv_full,
+                        kb * 64, u.g, krow);
+            tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128 + hb * 64 * 128, &map_v, &bars.kv_full,
+                        kb * 64, u.g, krow);
+          }
         }
         ++kv_fills;
         SlotWalk w;
@@ -355,7 +364,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
           if (use > 0) ok = mbar_wait(&bars.q_empty[st], (use - 1) & 1, wctx);
           if (!ok) break;
           const int32_t h = u.g * prm.G + w.e;
-          const int64_t rb = int64_t(w.r) * prm.B + u.b;
+          const int64_t rb = int64_t(w.r - prm.shard_begin) * prm.B + u.b;   // local (shard, b)
           const int32_t row0 = int32_t(rb * twoC + int64_t(w.i) * BQ);
           mbar_expect_tx(&bars.q_full[st], 2 * Cfg::QT_BYTES + 2 * BQ * 4);
           for (int kb = 0; kb < KB; ++kb) {
@@ -578,9 +587,9 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
         if (lane == 0) mbar_arrive(&bars.dq_empty);
         if (drow < HC) {
           const int32_t h = u.g * prm.G + w.e;
-          const int64_t row0 = (int64_t(w.r) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
+          const int64_t row0 = (int64_t(w.r - prm.shard_begin) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
           // head-major accumulator [Hq][rows][d]
-          float* base = prm.dq_acc + (int64_t(h) * prm.B * prm.S + row0) * HD + u.c * HC + drow;
+          float* base = prm.dq_acc + (int64_t(h) * prm.rows + row0) * HD + u.c * HC + drow;
           const int64_t rstride = HD;
 #pragma unroll
           for (int t = 0; t < BQ / 32; ++t)
@@ -705,13 +714,21 @@ __global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
       tc_fence_after();
       const uint32_t tAcc = tmem + (half == 0 ? Cfg::TM_DV : Cfg::TM_DK) + lane_addr;
       const float mul = half == 0 ? 1.0f : prm.scale;
-      __nv_bfloat16* dst = (half == 0 ? prm.dv : prm.dk) +
-                           ((int64_t(u.b) * prm.S + key) * prm.Hkv + u.g) * HD + u.c * HC;
+      const int64_t krow = kv_tensor_row(key, u.b, prm.S, prm.B, prm.D, prm.kv_shard_major);
+      __nv_bfloat16* dst = (half == 0 ? prm.dv : prm.dk) + (krow * prm.Hkv + u.g) * HD + u.c * HC;
+      // a key tile no query of the launch's shards sees has no MMA behind its
+      // accumulators: its dK / dV rows are zero
+      const bool empty = j == 0;
 #pragma unroll 1
       for (int c = 0; c < HC / 32; ++c) {
         uint32_t a[32];
-        tmem_ld32(tAcc + c * 32, a);
-        tmem_ld_wait();
+        if (!empty) {
+          tmem_ld32(tAcc + c * 32, a);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) a[e] = 0u;
+        }
         uint32_t o16[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
@@ -786,7 +803,8 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     zsa_bwd_wide_kernel(const __grid_constant__ CUtensorMap map_q,
                         const __grid_constant__ CUtensorMap map_k,
                         const __grid_constant__ CUtensorMap map_v,
-                        const __grid_constant__ CUtensorMap map_do, const BwdParams prm) {
+                        const __grid_constant__ CUtensorMap map_do,
+                        const __grid_constant__ CUtensorMap map_dq, const BwdParams prm) {
   using Cfg = BwdWideCfg<HD>;
   constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV;
   // the 128B-swizzled operand tiles need a 1024-byte aligned base; the shared-memory
@@ -809,7 +827,9 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     mbar_init(&bars.kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.q_full[s], 1);
-      mbar_init(&bars.q_empty[s], 1 + 8);   // MMA commit + 8 compute warps
+      // 8 compute warps (lse / Delta read) + 4 dQ warps (their reduce has read the
+      // dQ^T staged in this stage's Q / dO space, after every MMA of the slot)
+      mbar_init(&bars.q_empty[s], 8 + 4);
     }
     mbar_init(&bars.s_full, 1);
     mbar_init(&bars.p_full, 8);
@@ -838,6 +858,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     tma_prefetch_desc(&map_k);
     tma_prefetch_desc(&map_v);
     tma_prefetch_desc(&map_do);
+    tma_prefetch_desc(&map_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -865,10 +886,15 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
-        const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(u.n) * BKV);
-        for (int kb = 0; kb < KB; ++kb) {
-          tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128, &map_k, &bars.kv_full, kb * 64, u.g, key0);
-          tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128, &map_v, &bars.kv_full, kb * 64, u.g, key0);
+        for (int hb = 0; hb < BKV / 64; ++hb) {
+          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * 64, u.b, prm.S, prm.B, prm.D,
+                                             prm.kv_shard_major);
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128 + hb * 64 * 128, &map_k, &bars.kv_full,
+                        kb * 64, u.g, krow);
+            tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128 + hb * 64 * 128, &map_v, &bars.kv_full,
+                        kb * 64, u.g, krow);
+          }
         }
         ++kv_fills;
         SlotWalk w;
@@ -878,7 +904,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
           if (use > 0) ok = mbar_wait(&bars.q_empty[st], (use - 1) & 1, wctx);
           if (!ok) break;
           const int32_t h = u.g * prm.G + w.e;
-          const int64_t rb = int64_t(w.r) * prm.B + u.b;
+          const int64_t rb = int64_t(w.r - prm.shard_begin) * prm.B + u.b;   // local (shard, b)
           const int32_t row0 = int32_t(rb * twoC + int64_t(w.i) * BQ);
           mbar_expect_tx(&bars.q_full[st], 2 * Cfg::QT_BYTES + 2 * BQ * 4);
           for (int kb = 0; kb < KB; ++kb) {
@@ -1003,7 +1029,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
                      sdesc_sw128(sDS + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
             mma_commit(&bars.dq_full);
             mma_commit(&bars.dsm_free);
-            mma_commit(&bars.q_empty[st]);
+            // the stage's Q / dO are released by the dQ warps, which stage dQ^T there
           }
           ++q_it;
         }
@@ -1020,10 +1046,17 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     __syncwarp();
   } else if (warp >= Cfg::WARP_DQ) {
     // ------------------------------------------------------------ dQ warps
+    // dQ^T of a slot (TMEM lane = d index, column = q row) goes from TMEM to shared
+    // memory and from there into the fp32 accumulator by one TMA bulk reduce-add per
+    // warp: warp qw stages d rows 32qw .. 32qw+31 as a [128 q][32 d] fp32 box (128-byte
+    // rows, 128-byte swizzle).  The staging space is the slot's own Q and dO stage
+    // (HD * 512 bytes, exactly the size of dQ^T): once dQ^T is ready every MMA that reads
+    // that stage has completed, and the producer refills it only after the reduces have
+    // read it out (q_empty).  No per-element atomics leave the SM.
     const int qw = warp - Cfg::WARP_DQ;
-    const int drow = qw * 32 + lane;           // TMEM lane = d index of dQ^T
     const uint32_t tXT = tmem + Cfg::TM_XT + (uint32_t(qw * 32) << 16);
-    uint32_t dq_ph = 0;
+    const bool has_box = qw * 32 < HD;
+    uint32_t dq_ph = 0, q_it = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int slot = k % kUnitRing;
@@ -1040,32 +1073,47 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         dq_ph ^= 1;
         if (!ok) break;
         tc_fence_after();
-        const int32_t h = u.g * prm.G + w.e;
-        const int64_t row0 = (int64_t(w.r) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
-        // head-major accumulator [Hq][rows][d]: the slot's 128 rows are one 64 KB block
-        float* base = prm.dq_acc + (int64_t(h) * prm.B * prm.S + row0) * HD + drow;
-        const int64_t rstride = HD;
+        const int st = int(q_it & 1);
+        uint8_t* box = qw < KB ? smem + Cfg::SMEM_Q + st * Cfg::QT_BYTES + qw * (BQ * 128)
+                               : smem + Cfg::SMEM_DO + st * Cfg::QT_BYTES + (qw - KB) * (BQ * 128);
 #pragma unroll 1
-        for (int t = 0; t < BQ / 32; t += 2) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tXT + t * 32, v0);
-          tmem_ld32(tXT + (t + 1) * 32, v1);
+        for (int t = 0; t < BQ / 32; ++t) {
+          uint32_t v[32];
+          tmem_ld32(tXT + t * 32, v);
           tmem_ld_wait();
-          if (t + 2 == BQ / 32) {          // all of dQ^T read: XT may be overwritten
+          if (t + 1 == BQ / 32) {          // all of dQ^T read: XT may be overwritten
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.dq_empty);
           }
-          if (drow < HD) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) atomicAdd(base + (t * 32 + c) * rstride, __uint_as_float(v0[c]));
+          if (has_box) {
+            const uint32_t within = uint32_t(lane & 3) * 4;
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-              atomicAdd(base + ((t + 1) * 32 + c) * rstride, __uint_as_float(v1[c]));
+              *reinterpret_cast<uint32_t*>(box + sw128_offset(uint32_t(t * 32 + c), uint32_t(lane >> 2)) +
+                                           within) = v[c];
           }
         }
+        if (has_box) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int32_t h = u.g * prm.G + w.e;
+            const int32_t row0 =
+                int32_t((int64_t(w.r - prm.shard_begin) * prm.B + u.b) * twoC + int64_t(w.i) * BQ);
+            tma_reduce_add_3d(&map_dq, box, qw * 32, row0, h);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.q_empty[st]);
+        ++q_it;
       }
     }
+    // every reduce issued by this warp has been performed before the kernel ends
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ compute warps
     // group h = warp / 4 handles q rows 64h .. 64h+63 of every slot (contiguous
@@ -1080,6 +1128,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     uint32_t q_it = 0, s_ph = 0, dp_ph = 0, acc_ph = 0, dsm_uses = 0;
     uint32_t q_full_uses[2] = {0, 0};
     bool ok = true;
+    int nslots = 0;                            // slots of the current unit
     for (int k = 0; ok; ++k) {
       const int slot = k % kUnitRing;
       ok = warp_wait_b(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
@@ -1091,7 +1140,9 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
       const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
       const int64_t key = int64_t(u.n) * BKV + row;
       SlotWalk w;
+      nslots = 0;
       for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
+        ++nslots;
         const int st = int(q_it & 1);
         ok = warp_wait_b(&bars.q_full[st], q_full_uses[st] & 1, wctx);
         ++q_full_uses[st];
@@ -1171,13 +1222,21 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
       tc_fence_after();
       const uint32_t tAcc = tmem + (hgrp == 0 ? Cfg::TM_DV : Cfg::TM_DK) + lane_addr;
       const float mul = hgrp == 0 ? 1.0f : prm.scale;
-      __nv_bfloat16* dst = (hgrp == 0 ? prm.dv : prm.dk) +
-                           ((int64_t(u.b) * prm.S + key) * prm.Hkv + u.g) * HD;
+      const int64_t krow = kv_tensor_row(key, u.b, prm.S, prm.B, prm.D, prm.kv_shard_major);
+      __nv_bfloat16* dst = (hgrp == 0 ? prm.dv : prm.dk) + (krow * prm.Hkv + u.g) * HD;
+      // a key tile no query of the launch's shards sees has no MMA behind its
+      // accumulators: its dK / dV rows are zero
+      const bool empty = nslots == 0;
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t a[32];
-        tmem_ld32(tAcc + c * 32, a);
-        tmem_ld_wait();
+        if (!empty) {
+          tmem_ld32(tAcc + c * 32, a);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) a[e] = 0u;
+        }
         uint32_t o16[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
@@ -1214,8 +1273,8 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   constexpr int kChunks = kWide ? 1 : HD / 128;    // d chunks of 128 per key tile
   // the 128-row kernel aligns its dynamic shared memory itself (no slack needed)
   constexpr int kSmem = kWide ? Cfg::SMEM_BYTES : Cfg::SMEM_BYTES + 1024;
-  const int64_t rows = a.S * a.B;             // shard-major rows (D * B * 2C)
   const int64_t twoC = a.S / a.D;
+  const int64_t rows = int64_t(a.shard_count) * a.B * twoC;   // local shard-major rows
   const int sms = num_sms();
   // K2: Delta and a zeroed dQ accumulator
   {
@@ -1245,9 +1304,16 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), uint64_t(a.B * a.S)};
     const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hkv) * HD * 2};
-    const uint32_t box[3] = {64, 1, uint32_t(Cfg::BKV)};
+    const uint32_t box[3] = {64, 1, 64};   // 64-key boxes: one zigzag chunk each
     if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
     if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
+  }
+  CUtensorMap mdq;
+  if constexpr (kWide) {
+    const uint64_t dims[3] = {uint64_t(HD), uint64_t(rows), uint64_t(a.Hq)};
+    const uint64_t strides[2] = {uint64_t(HD) * 4, uint64_t(rows) * HD * 4};
+    const uint32_t box[3] = {32, uint32_t(Cfg::BQ), 1};
+    if (!make_map_f32_sw128(&mdq, a.dq_acc, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
   BwdParams p;
   p.lse = a.lse;
@@ -1263,6 +1329,10 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.n_chunks = kChunks;
   p.bq = Cfg::BQ;
   p.n_ktiles = int32_t(a.S / Cfg::BKV);
+  p.kv_shard_major = a.kv_layout;
+  p.shard_begin = a.shard_begin;
+  p.shard_end = a.shard_begin + a.shard_count;
+  p.rows = rows;
   p.counter = a.status + 32;
   p.scale = a.scale;
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
@@ -1281,7 +1351,10 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   const int grid = p.n_units < sms ? p.n_units : sms;
   const TraceEvents tr = trace_events(2);
   if (tr.begin) cudaEventRecord(tr.begin, stream);
-  kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, p);
+  if constexpr (kWide)
+    kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
+  else
+    kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, p);
   cudaError_t e = cudaGetLastError();
   if (tr.end) cudaEventRecord(tr.end, stream);
   if (e != cudaSuccess) return int(e);

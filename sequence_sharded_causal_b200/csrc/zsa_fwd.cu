@@ -73,6 +73,8 @@ struct FwdParams {
   float* lse;
   int64_t S, C;
   int32_t B, Hq, Hkv, D, causal;
+  int32_t kv_shard_major;  // K/V rows in the shard-major zigzag order instead of position order
+  int32_t shard_begin;     // first shard this launch computes (Q-layout rows are local)
   float scale_log2;
   int* status;
   int* counter;       // next unclaimed unit (zeroed before every launch)
@@ -204,7 +206,8 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
           if (q_fills[s] > 0) ok = mbar_wait(&bars.q_empty[s], (q_fills[s] - 1) & 1, wctx);
           if (!ok) break;
           mbar_expect_tx(&bars.q_full[s], Cfg::Q_BYTES);
-          const int32_t row0 = int32_t((int64_t(u.r) * prm.B + u.b) * twoC + int64_t(u.tile[s]) * 128);
+          const int32_t row0 =
+              int32_t((int64_t(u.r - prm.shard_begin) * prm.B + u.b) * twoC + int64_t(u.tile[s]) * 128);
           for (int kb = 0; kb < KB; ++kb)
             tma_load_3d(smem + Cfg::SMEM_Q + s * Cfg::Q_BYTES + kb * 128 * 128, &map_q,
                         &bars.q_full[s], kb * 64, u.head[s], row0);
@@ -217,26 +220,32 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             const uint32_t it = kv_it + uint32_t(n);
             const int st = int(it % ST);
             const uint32_t use = it / ST;
-            const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(n) * BK);
             if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.k_full[st], Cfg::KV_BYTES);
-            for (int kb = 0; kb < KB; ++kb)
-              tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128, &map_k,
-                          &bars.k_full[st], kb * 64, u.g, key0);
+            for (int hb = 0; hb < BK / 64; ++hb) {
+              const int32_t krow = kv_tensor_row(int64_t(n) * BK + hb * 64, u.b, prm.S, prm.B,
+                                                 prm.D, prm.kv_shard_major);
+              for (int kb = 0; kb < KB; ++kb)
+                tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
+                            &map_k, &bars.k_full[st], kb * 64, u.g, krow);
+            }
             ++k_fills[st];
           }
           if (n >= 1) {
             const uint32_t it = kv_it + uint32_t(n - 1);
             const int st = int(it % ST);
             const uint32_t use = it / ST;
-            const int32_t key0 = int32_t(int64_t(u.b) * prm.S + int64_t(n - 1) * BK);
             if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.v_full[st], Cfg::KV_BYTES);
-            for (int kb = 0; kb < KB; ++kb)
-              tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128, &map_v,
-                          &bars.v_full[st], kb * 64, u.g, key0);
+            for (int hb = 0; hb < BK / 64; ++hb) {
+              const int32_t vrow = kv_tensor_row(int64_t(n - 1) * BK + hb * 64, u.b, prm.S, prm.B,
+                                                 prm.D, prm.kv_shard_major);
+              for (int kb = 0; kb < KB; ++kb)
+                tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
+                            &map_v, &bars.v_full[st], kb * 64, u.g, vrow);
+            }
             ++v_fills[st];
           }
         }
@@ -492,7 +501,8 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const float inv_l = 1.0f / r_run;
-      const int64_t grow = (int64_t(u.r) * prm.B + u.b) * twoC + j;    // shard-major row
+      const int64_t rb = int64_t(u.r - prm.shard_begin) * prm.B + u.b;   // local (shard, b)
+      const int64_t grow = rb * twoC + j;                                 // shard-major row
       __nv_bfloat16* orow_g = prm.o + (grow * prm.Hq + u.head[s]) * HD;
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
@@ -509,7 +519,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         for (int v4 = 0; v4 < 4; ++v4)
           dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
       }
-      prm.lse[((int64_t(u.r) * prm.B + u.b) * prm.Hq + u.head[s]) * twoC + j] =
+      prm.lse[(rb * prm.Hq + u.head[s]) * twoC + j] =
           (m_run + log2f(l_run)) * 0.69314718055994530942f;
       tc_fence_before();
       __syncwarp();
@@ -526,7 +536,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
 template <int HD>
 int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   using Cfg = FwdCfg<HD>;
-  const int64_t rows = a.S * a.B;  // D * B * 2C shard-major rows
+  const int64_t rows = int64_t(a.shard_count) * a.B * (a.S / a.D);  // local shard-major rows
   CUtensorMap mq, mk, mv;
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hq), uint64_t(rows)};
@@ -537,7 +547,7 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), uint64_t(a.B * a.S)};
     const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hkv) * HD * 2};
-    const uint32_t box[3] = {64, 1, uint32_t(Cfg::BK)};
+    const uint32_t box[3] = {64, 1, 64};   // 64-key boxes: one zigzag chunk each
     if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
     if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
@@ -549,6 +559,8 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   p.S = a.S;
   p.C = a.S / (2 * int64_t(a.D));
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.D = a.D; p.causal = a.causal;
+  p.kv_shard_major = a.kv_layout;
+  p.shard_begin = a.shard_begin;
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
   p.status = a.status;
   p.counter = a.status + 32;

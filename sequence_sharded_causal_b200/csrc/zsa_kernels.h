@@ -18,6 +18,9 @@ struct FwdArgs {
   int64_t S;
   int32_t B, Hq, Hkv, d, D, causal;
   float scale;
+  int32_t kv_layout;       // 0: K/V [B][S][Hkv][d]; 1: shard-major [D][B][2C][Hkv][d]
+  int32_t shard_begin;     // the call computes the queries of shards
+  int32_t shard_count;     //   [shard_begin, shard_begin + shard_count)
   int* status;
   uint64_t wait_limit_ns;
   int inject_stall;        // test hook: the MMA threads first wait on a barrier nobody arrives at
@@ -33,14 +36,28 @@ struct BwdArgs {
   void* dq;
   void* dk;
   void* dv;
-  float* delta;            // [D][B][Hq][2C] workspace
-  float* dq_acc;           // [Hq][D*B*2C][d] workspace (head-major)
+  float* delta;            // [shards][B][Hq][2C] workspace
+  float* dq_acc;           // [Hq][shards*B*2C][d] workspace (head-major)
   int64_t S;
   int32_t B, Hq, Hkv, d, D, causal;
   float scale;
+  int32_t kv_layout;       // as in FwdArgs; dK / dV are written in the same layout
+  int32_t shard_begin, shard_count;
   int* status;
   uint64_t wait_limit_ns;
   int inject_stall;        // test hook: the MMA threads first wait on a barrier nobody arrives at
+};
+
+// Partial results to merge (ring attention): n parts of the Q layout (bf16 O) and the
+// lse layout (fp32), rows = local Q-layout rows of the problem.
+constexpr int kMergeMaxParts = 32;
+struct MergeArgs {
+  const void* o[kMergeMaxParts];
+  const float* lse[kMergeMaxParts];
+  void* o_out;
+  float* lse_out;
+  int64_t S, rows;
+  int32_t Hq, d, D, n;
 };
 
 // Tiling the forward kernel is built for, per head dim.
@@ -54,7 +71,7 @@ inline void fwd_tiling(int d, int32_t* bq, int32_t* bk, int32_t* slots) {
 struct TraceEvents {
   cudaEvent_t begin, end;
 };
-TraceEvents trace_events(int which);  // which: 0 fwd, 1 bwd pre, 2 bwd main, 3 dQ convert
+TraceEvents trace_events(int which);  // 0 fwd, 1 bwd pre, 2 bwd main, 3 dQ convert, 4 merge
 
 // Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once
 // per (kernel, device): cudaFuncSetAttribute applies to the device current at the time
@@ -69,5 +86,6 @@ int inject_stall();
 // Returns a cudaError_t (cudaSuccess on success).
 int launch_fwd(const FwdArgs& a, cudaStream_t stream);
 int launch_bwd(const BwdArgs& a, cudaStream_t stream);
+int launch_merge(const MergeArgs& a, cudaStream_t stream);
 
 }  // namespace zsa

@@ -95,7 +95,9 @@ extern "C" int zsa_attn_bwd_noalloc(const zsa_problem* problem, const void* q, c
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   uint8_t* base = static_cast<uint8_t*>(scratch);
   if (cudaMemsetAsync(base, 0, kNoAllocStatusBytes, stream) != cudaSuccess) return ZSA_ERR_CUDA;
-  const size_t stats = size_t(problem->B) * problem->S * problem->Hq * sizeof(float);
+  const int32_t shards = problem->shard_count ? problem->shard_count : problem->D;
+  const size_t stats =
+      size_t(shards) * problem->B * (problem->S / problem->D) * problem->Hq * sizeof(float);
   zsa::BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
   a.dq = dq; a.dk = dk; a.dv = dv;
@@ -104,6 +106,9 @@ extern "C" int zsa_attn_bwd_noalloc(const zsa_problem* problem, const void* q, c
   a.S = problem->S; a.B = int32_t(problem->B); a.Hq = problem->Hq; a.Hkv = problem->Hkv;
   a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
   a.scale = problem->softmax_scale;
+  a.kv_layout = problem->kv_layout;
+  a.shard_begin = problem->shard_begin;
+  a.shard_count = shards;
   a.status = reinterpret_cast<int*>(base);
   a.wait_limit_ns = zsa::wait_limit_ns();
   a.inject_stall = zsa::inject_stall();

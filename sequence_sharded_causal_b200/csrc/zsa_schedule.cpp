@@ -13,8 +13,10 @@
 namespace zsa {
 
 bool build_schedule(int64_t S, int32_t D, int32_t B, int32_t Hq, int32_t Hkv, int32_t causal,
-                    int32_t bq, int32_t bk, int32_t slots, Schedule* out) {
+                    int32_t bq, int32_t bk, int32_t slots, int32_t shard_begin,
+                    int32_t shard_count, Schedule* out) {
   if (S <= 0 || D <= 0 || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return false;
+  if (shard_begin < 0 || shard_count <= 0 || shard_begin + shard_count > D) return false;
   if (bq <= 0 || bk <= 0 || (slots != 1 && slots != 2)) return false;
   if (S % (2 * int64_t(D)) != 0 || (S / D) % bq != 0 || S % bk != 0) return false;
   const int64_t C = S / (2 * int64_t(D));
@@ -31,6 +33,7 @@ bool build_schedule(int64_t S, int32_t D, int32_t B, int32_t Hq, int32_t Hkv, in
 
   out->S = S; out->D = D; out->B = B; out->Hq = Hq; out->Hkv = Hkv;
   out->causal = causal; out->bq = bq; out->bk = bk; out->slots = slots;
+  out->shard_begin = shard_begin; out->shard_count = shard_count;
   out->shard_tiles.assign(size_t(D), 0);
   for (int32_t r = 0; r < D; ++r) {
     int64_t w = 0;
@@ -44,10 +47,10 @@ bool build_schedule(int64_t S, int32_t D, int32_t B, int32_t Hq, int32_t Hkv, in
   };
   const int64_t runs = (T * G + slots - 1) / slots;
   std::vector<Keyed> list;
-  list.reserve(size_t(int64_t(B) * Hkv * D * runs));
+  list.reserve(size_t(int64_t(B) * Hkv * shard_count * runs));
   for (int32_t b = 0; b < B; ++b)
     for (int32_t g = 0; g < Hkv; ++g)
-      for (int32_t r = 0; r < D; ++r)
+      for (int32_t r = shard_begin; r < shard_begin + shard_count; ++r)
         for (int64_t m = 0; m < runs; ++m) {
           Keyed x;
           const int64_t s0 = m * slots, s1 = s0 + 1;

@@ -28,11 +28,12 @@ inline EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// bf16 tensor of `rank` dims (dim 0 innermost, contiguous); strides in BYTES for dims
-// 1..rank-1; box in elements; 128-byte swizzle (box dim 0 must be 64 bf16 = 128 B).
-inline bool make_map_bf16_sw128(CUtensorMap* map, const void* base, int rank,
-                                const uint64_t* dims, const uint64_t* strides_bytes,
-                                const uint32_t* box) {
+// Tensor of `rank` dims (dim 0 innermost, contiguous) with elements of `dtype`; strides
+// in BYTES for dims 1..rank-1; box in elements; 128-byte swizzle (box dim 0 must span
+// 128 bytes: 64 bf16 or 32 fp32).
+inline bool make_map_sw128(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                           int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                           const uint32_t* box) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   cuuint64_t gdim[5];
@@ -45,10 +46,24 @@ inline bool make_map_bf16_sw128(CUtensorMap* map, const void* base, int rank,
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) gstr[i] = strides_bytes[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                  gdim, gstr, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), gdim, gstr, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+inline bool make_map_bf16_sw128(CUtensorMap* map, const void* base, int rank,
+                                const uint64_t* dims, const uint64_t* strides_bytes,
+                                const uint32_t* box) {
+  return make_map_sw128(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes,
+                        box);
+}
+
+inline bool make_map_f32_sw128(CUtensorMap* map, const void* base, int rank,
+                               const uint64_t* dims, const uint64_t* strides_bytes,
+                               const uint32_t* box) {
+  return make_map_sw128(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, rank, dims, strides_bytes,
+                        box);
 }
 
 }  // namespace zsa

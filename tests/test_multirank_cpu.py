@@ -1,8 +1,9 @@
 """The N > 1 host path of bench.py on CPU: two gloo ranks.
 
-With more than one GPU the single-GPU path runs as independent replicas (it has no
-exchange step); what spans ranks is the timing rule -- the job's time is the slowest
-rank's -- and the whole-job value, the sum of every rank's work over that time.
+With more than one GPU each rank runs its share of one problem (its own zigzag shards;
+the collectives are covered by tests/test_sharded_cpu.py); what spans ranks in the
+bench is the timing rule -- the job's time is the slowest rank's -- and the whole-job
+value, the sum of every rank's work over that time.
 """
 import os
 import socket

@@ -40,6 +40,13 @@ MUTANTS = {
     "kend_off_by_one": ("return largest / bk + 1;", "return largest / bk;"),
     "order_ascending": ("return a->key_work > b->key_work ? -1 : 1;",
                         "return a->key_work < b->key_work ? -1 : 1;"),
+    "keys_diagonal_dropped": ("if (causal && p + 1 < end) end = p + 1;",
+                              "if (causal && p < end) end = p;"),
+    "keys_range_shifted": ("for (int64_t key = key_lo; key < end; ++key)",
+                           "for (int64_t key = key_lo + (key_lo > 0); key < end; ++key)"),
+    "merge_weights_unnormalised": ("double w = exp(lse_parts[(int64_t)i * m + x] - lse_x);",
+                                   "double w = exp(lse_parts[(int64_t)i * m + x] - mx);"),
+    "merge_lse_max_dropped": ("double lse_x = mx + log(l);", "double lse_x = log(l);"),
 }
 
 
@@ -111,6 +118,25 @@ def _pins_pass():
     dq_nat = inputs.to_shard_major(torch.from_numpy(dq_ref), perm, D).numpy().reshape(-1, Hq, d)
     if np.abs(dq_rows - dq_nat[rows]).max() > 1e-11:
         return False
+    # key-range forward vs the masked brute force, and the merge of a split
+    S2, D2 = 32, 2
+    perm2, _ = oracle.partition(S2, D2)
+    qk = rng.standard_normal((1, S2, 2, 8))
+    kk = rng.standard_normal((1, S2, 1, 8))
+    vk = rng.standard_normal((1, S2, 1, 8))
+    qs2 = inputs.to_shard_major(torch.from_numpy(qk), perm2, D2).numpy()
+    for lo, hi in ((5, 20), (11, 32)):
+        ok_, lk = oracle.attn_fwd_keys(qs2, kk, vk, D2, lo, hi)
+        o_b, l_b = brute.key_range_attention(qk, kk, vk, lo, hi)
+        o_n = inputs.from_shard_major(torch.from_numpy(ok_), perm2).numpy()
+        if np.abs(o_n - o_b).max() > 1e-12:
+            return False
+    o_f, l_f = oracle.attn_fwd(qs2, kk, vk, D2)
+    pa = oracle.attn_fwd_keys(qs2, kk, vk, D2, 0, 13)
+    pb = oracle.attn_fwd_keys(qs2, kk, vk, D2, 13, 32)
+    o_m, l_m = oracle.attn_merge([pa[0], pb[0]], [pa[1], pb[1]])
+    if np.abs(o_m - o_f).max() > 1e-12 or np.abs(l_m - l_f).max() > 1e-12:
+        return False
     return True
 
 
@@ -125,7 +151,8 @@ def test_mutant_is_caught(tmp_path, name, monkeypatch):
     real = oracle._load()
     mutant = ctypes.CDLL(lib_path)
     for fn in ("oracle_partition", "oracle_schedule", "oracle_attn_fwd", "oracle_attn_fwd_rows",
-               "oracle_attn_bwd", "oracle_attn_dq_rows"):
+               "oracle_attn_bwd", "oracle_attn_dq_rows", "oracle_attn_fwd_keys",
+               "oracle_attn_merge"):
         getattr(mutant, fn).argtypes = getattr(real, fn).argtypes
         getattr(mutant, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", mutant)
