@@ -38,16 +38,16 @@
 //   * one MMA-issuing thread; 8 compute warps; 4 dQ warps as above.
 #include <cuda_bf16.h>
 
-#include <type_traits>
 
+#include "zsa_bwd_common.cuh"
 #include "zsa_kernels.h"
 #include "zsa_ptx.cuh"
 #include "zsa_tma_host.h"
 
 namespace zsa {
 namespace {
+using namespace bwd;
 
-constexpr float kLog2e = 1.4426950408889634f;
 
 // ------------------------------------------------------------------ K2: Delta + zero dQacc
 template <int HD>
@@ -118,636 +118,6 @@ __global__ void __launch_bounds__(256) zsa_dq_convert_kernel(const float* __rest
       reinterpret_cast<uint4*>(dq + row * int64_t(Hq) * HD)[t] = r;
     }
   }
-}
-
-// ------------------------------------------------------------------ K3: main backward
-template <int HD>
-struct BwdCfg {
-  static constexpr int BKV = 128;                   // keys per CTA tile (TMEM lanes)
-  static constexpr int BQ = HD == 256 ? 32 : 64;    // query rows per slot
-  static constexpr int HC = HD == 256 ? 128 : HD;   // d columns one unit accumulates (dK, dV)
-  static constexpr int NCHUNK = HD / HC;            // units per key tile
-  static constexpr int KB = HD / 64;                // 64-wide d blocks of K, V, Q, dO
-  static constexpr int CB = HC / 64;                // 64-wide d blocks per chunk
-  static constexpr int HALF = BQ / 2;               // slot columns per compute group
-  // dS for the dQ MMA: MN-major [keys][BQ] (BQ = 64, one 128-byte swizzle row per key)
-  // or K-major [BQ][keys] (BQ = 32)
-  static constexpr bool DS_KMAJOR = BQ < 64;
-  static constexpr int NQST = 2;    // Q/dO stages
-  static constexpr int KV_BYTES = BKV * HD * 2;          // K (or V) tile
-  static constexpr int QT_BYTES = BQ * HD * 2;           // Q (or dO) slot tile
-  static constexpr int DS_BYTES = BKV * BQ * 2;          // dS^T tile (bf16)
-  static constexpr int SMEM_K = 0;
-  static constexpr int SMEM_V = SMEM_K + KV_BYTES;
-  static constexpr int SMEM_Q = SMEM_V + KV_BYTES;
-  static constexpr int SMEM_DO = SMEM_Q + NQST * QT_BYTES;
-  static constexpr int SMEM_DS = SMEM_DO + NQST * QT_BYTES;
-  static constexpr int SMEM_LSE = SMEM_DS + 2 * DS_BYTES;      // [NQST][BQ] fp32
-  static constexpr int SMEM_DELTA = SMEM_LSE + NQST * BQ * 4;  // [NQST][BQ] fp32
-  static constexpr int SMEM_BYTES = SMEM_DELTA + NQST * BQ * 4;
-  static constexpr int WARP_DQ = 8;       // warps 8..11
-  static constexpr int WARP_LOAD = 12;
-  static constexpr int WARP_MMA = 13;
-  static constexpr int NTHREADS = 14 * 32;
-  static constexpr uint32_t TM_DV = 0;
-  static constexpr uint32_t TM_DK = HC;
-  static constexpr uint32_t TM_ST = 2 * HC;             // two buffers of BQ columns
-  static constexpr uint32_t TM_DPT = 2 * HC + 2 * BQ;
-  static constexpr uint32_t TM_DQT = 2 * HC + 3 * BQ;
-  static constexpr uint32_t TM_COLS = 512;
-  static_assert(2 * HC + 4 * BQ <= 512, "TMEM budget");
-  static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
-};
-
-struct BwdParams {
-  const float* lse;
-  const float* delta;
-  float* dq_acc;
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
-  int64_t S, C;
-  int32_t B, Hq, Hkv, G, D, causal;
-  int32_t n_units, n_qtiles;  // n_qtiles = BQ-row tiles per shard
-  int32_t n_chunks, bq;       // d chunks per key tile, query rows per slot
-  int32_t n_ktiles;           // S / 128
-  int32_t kv_shard_major;     // K/V/dK/dV rows in the shard-major zigzag order
-  int32_t shard_begin, shard_end;   // the launch computes the queries of these shards
-  int64_t rows;               // local Q-layout rows: (shard_end - shard_begin) * B * 2C
-  float scale, scale_log2;
-  int* status;
-  int* counter;       // next unclaimed unit (zeroed before every launch)
-  uint64_t wait_limit_ns;
-  int inject_stall;
-};
-
-constexpr int kUnitRing = 4;   // claimed units in flight between the producer and the others
-
-struct BwdBars {
-  uint64_t kv_full, kv_empty;
-  uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], st_free[2];
-  uint64_t dp_full, dpt_free;
-  uint64_t p_full, ds_full;
-  uint64_t dsm_free[2];
-  uint64_t dq_full, dq_empty;
-  uint64_t acc_full, acc_empty;
-  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
-  uint64_t drain, never;
-};
-
-// One key tile of work.
-struct KvUnit {
-  int32_t n, b, g, c;   // key tile, batch, kv head, d chunk
-};
-
-// Units are claimed dynamically in the order (b, kv head g, key tile n, d chunk c):
-// CTAs busy at the same time work on one head group, sharing its Q / dO stream and
-// its dQ accumulator rows in L2; within a group n ascends, i.e. the work per unit
-// (the number of q tiles that see key tile n) descends, so each group ends with its
-// shortest units.
-__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int Hkv, int NT, int NC) {
-  KvUnit u;
-  u.c = idx % NC;
-  u.n = (idx / NC) % NT;
-  u.g = (idx / (NC * NT)) % Hkv;
-  u.b = idx / (NC * NT * Hkv);
-  return u;
-}
-
-// Enumerates the q slots (shard r, BQ-row tile i, head offset e) that see key tile n,
-// in (r, i, e) order.  Every role walks the same sequence.  A BQ-row tile never
-// straddles a zigzag chunk (C is a multiple of 64), so its positions are contiguous.
-struct SlotWalk {
-  int32_t r, i, e;
-  int64_t p0;   // position of the tile's first row (its rows are p0 .. p0+BQ-1)
-};
-
-__device__ __forceinline__ int64_t zz_pos(int64_t C, int32_t D, int32_t r, int64_t j) {
-  return j < C ? int64_t(r) * C + j : int64_t(2 * D - 1 - r) * C + (j - C);
-}
-
-__device__ __forceinline__ bool tile_sees(const BwdParams& p, int32_t r, int32_t i, int32_t n,
-                                          int64_t* p0) {
-  *p0 = zz_pos(p.C, p.D, r, int64_t(i) * p.bq);
-  // positions rise along a shard, so the tile's last row holds its largest position
-  return !p.causal || (zz_pos(p.C, p.D, r, int64_t(i) * p.bq + p.bq - 1) >= int64_t(n) * 128);
-}
-
-// First slot at or after (r, i, 0); false when the walk is over.  Only the launch's
-// shards [shard_begin, shard_end) are walked.
-__device__ __forceinline__ bool walk_seek(const BwdParams& p, int32_t n, SlotWalk& w) {
-  while (w.r < p.shard_end) {
-    if (tile_sees(p, w.r, w.i, n, &w.p0)) return true;
-    if (++w.i == p.n_qtiles) {
-      w.i = 0;
-      ++w.r;
-    }
-  }
-  return false;
-}
-__device__ __forceinline__ bool walk_first(const BwdParams& p, int32_t n, SlotWalk& w) {
-  w.r = p.shard_begin; w.i = 0; w.e = 0;
-  return walk_seek(p, n, w);
-}
-__device__ __forceinline__ bool walk_next(const BwdParams& p, int32_t n, SlotWalk& w) {
-  if (++w.e < p.G) return true;
-  w.e = 0;
-  if (++w.i == p.n_qtiles) {
-    w.i = 0;
-    ++w.r;
-  }
-  return walk_seek(p, n, w);
-}
-
-__device__ __forceinline__ bool warp_wait_b(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  bool ok = mbar_wait(bar, parity, w);
-  return __all_sync(0xffffffffu, ok);
-}
-
-template <int HD>
-__global__ void __launch_bounds__(BwdCfg<HD>::NTHREADS, 1)
-    zsa_bwd_kernel(const __grid_constant__ CUtensorMap map_q,
-                   const __grid_constant__ CUtensorMap map_k,
-                   const __grid_constant__ CUtensorMap map_v,
-                   const __grid_constant__ CUtensorMap map_do, const BwdParams prm) {
-  using Cfg = BwdCfg<HD>;
-  constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV, HC = Cfg::HC, CB = Cfg::CB;
-  constexpr int HALF = Cfg::HALF;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  __shared__ BwdBars bars;
-  __shared__ uint32_t tmem_base_s;
-  __shared__ int abort_s;
-  __shared__ int unit_ring[kUnitRing];
-
-  const int warp = int(warp_id()), lane = int(lane_id());
-  if (threadIdx.x == 0) {
-    abort_s = 0;
-    mbar_init(&bars.kv_full, 1);
-    mbar_init(&bars.kv_empty, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.q_full[s], 1);
-      mbar_init(&bars.q_empty[s], 1 + 8);   // MMA commit + 8 compute warps
-      mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.st_free[s], 1);
-      mbar_init(&bars.dsm_free[s], 1);
-    }
-    mbar_init(&bars.dp_full, 1);
-    mbar_init(&bars.dpt_free, 1);
-    mbar_init(&bars.p_full, 8);
-    mbar_init(&bars.ds_full, 8);
-    mbar_init(&bars.dq_full, 1);
-    mbar_init(&bars.dq_empty, 4);
-    mbar_init(&bars.acc_full, 1);
-    mbar_init(&bars.acc_empty, 8);
-    for (int s = 0; s < kUnitRing; ++s) {
-      mbar_init(&bars.unit_full[s], 1);
-      mbar_init(&bars.unit_empty[s], 1 + 8 + 4);   // MMA thread + compute + dQ warps
-    }
-    mbar_init(&bars.drain, 1);
-    mbar_init(&bars.never, 1);
-    fence_mbar_init();
-  }
-  if (warp == Cfg::WARP_MMA) {
-    tmem_alloc(&tmem_base_s, Cfg::TM_COLS);
-    tmem_relinquish();
-  }
-  if (warp == Cfg::WARP_LOAD && lane == 0) {
-    tma_prefetch_desc(&map_q);
-    tma_prefetch_desc(&map_k);
-    tma_prefetch_desc(&map_v);
-    tma_prefetch_desc(&map_do);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base_s;
-  const WaitCtx wctx{&abort_s, prm.status, prm.wait_limit_ns};
-  const int64_t twoC = 2 * prm.C;
-
-  if (warp == Cfg::WARP_LOAD) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t q_it = 0, kv_fills = 0;
-      uint32_t q_fills[2] = {0, 0};
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        // claim the next unit and hand it to the other roles through the ring
-        const int slot = k % kUnitRing;
-        if (k >= kUnitRing) ok = mbar_wait(&bars.unit_empty[slot], ((k / kUnitRing) - 1) & 1, wctx);
-        if (!ok) break;
-        int idx = atomicAdd(prm.counter, 1);
-        if (idx >= prm.n_units) idx = -1;
-        unit_ring[slot] = idx;
-        mbar_arrive(&bars.unit_full[slot]);
-        if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
-        if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
-        if (!ok) break;
-        mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
-        for (int hb = 0; hb < BKV / 64; ++hb) {
-          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * 64, u.b, prm.S, prm.B, prm.D,
-                                             prm.kv_shard_major);
-          for (int kb = 0; kb < KB; ++kb) {
-            tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128 + hb * 64 * 128, &map_k, &bars.kv_full,
-                        kb * 64, u.g, krow);
-            tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128 + hb * 64 * 128, &map_v, &bars.kv_full,
-                        kb * 64, u.g, krow);
-          }
-        }
-        ++kv_fills;
-        SlotWalk w;
-        for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
-          const int st = int(q_it & 1);
-          const uint32_t use = q_it >> 1;
-          if (use > 0) ok = mbar_wait(&bars.q_empty[st], (use - 1) & 1, wctx);
-          if (!ok) break;
-          const int32_t h = u.g * prm.G + w.e;
-          const int64_t rb = int64_t(w.r - prm.shard_begin) * prm.B + u.b;   // local (shard, b)
-          const int32_t row0 = int32_t(rb * twoC + int64_t(w.i) * BQ);
-          mbar_expect_tx(&bars.q_full[st], 2 * Cfg::QT_BYTES + 2 * BQ * 4);
-          for (int kb = 0; kb < KB; ++kb) {
-            tma_load_3d(smem + Cfg::SMEM_Q + st * Cfg::QT_BYTES + kb * BQ * 128, &map_q,
-                        &bars.q_full[st], kb * 64, h, row0);
-            tma_load_3d(smem + Cfg::SMEM_DO + st * Cfg::QT_BYTES + kb * BQ * 128, &map_do,
-                        &bars.q_full[st], kb * 64, h, row0);
-          }
-          const int64_t stat = (rb * prm.Hq + h) * twoC + int64_t(w.i) * BQ;
-          bulk_load(smem + Cfg::SMEM_LSE + st * BQ * 4, prm.lse + stat, BQ * 4, &bars.q_full[st]);
-          bulk_load(smem + Cfg::SMEM_DELTA + st * BQ * 4, prm.delta + stat, BQ * 4, &bars.q_full[st]);
-          ++q_fills[st];
-          ++q_it;
-        }
-      }
-      if (!ok) {
-        const uint64_t lim = 1000000000ull;
-        if (kv_fills > 0) mbar_drain(&bars.kv_full, (kv_fills - 1) & 1, lim);
-        for (int s = 0; s < 2; ++s)
-          if (q_fills[s] > 0) mbar_drain(&bars.q_full[s], (q_fills[s] - 1) & 1, lim);
-      }
-    }
-  } else if (warp == Cfg::WARP_MMA) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16(128, BQ, false, false);
-      const uint32_t idesc_kv = idesc_bf16(128, HC, false, true);
-      const uint32_t idesc_dq = idesc_bf16(128, BQ, true, !Cfg::DS_KMAJOR);
-      const uint32_t sK = smem_u32(smem + Cfg::SMEM_K);
-      const uint32_t sV = smem_u32(smem + Cfg::SMEM_V);
-      const uint32_t sQ = smem_u32(smem + Cfg::SMEM_Q);
-      const uint32_t sDO = smem_u32(smem + Cfg::SMEM_DO);
-      const uint32_t sDS = smem_u32(smem + Cfg::SMEM_DS);
-      // dQ^T = K^T dS^T: A = K^T, M = d in 64-row blocks at the d-block stride of the K
-      // tile.  With d = 64 the second M block points at V (its rows are never read).
-      const uint32_t lbo_kt = HD >= 128 ? uint32_t(BKV * 128) : uint32_t(Cfg::SMEM_V - Cfg::SMEM_K);
-      uint32_t kv_ph = 0, q_it = 0;
-      uint32_t q_full_uses[2] = {0, 0};
-      uint32_t p_ph = 0, ds_ph = 0;
-      uint32_t st_commits[2] = {0, 0}, st_waits[2] = {0, 0};
-      uint32_t dpt_commits = 0, dpt_waits = 0;
-      uint32_t dq_commits = 0, dq_waits = 0;
-      uint32_t acc_commits = 0;
-      bool ok = true;
-      if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
-      // TMEM column (bf16 pairs) of q columns 16ks .. 16ks+15 of P^T / dS^T: compute
-      // group h writes its HALF columns as HALF/2 packed columns at h*HALF
-      auto p_col = [](int ks) -> uint32_t {
-        return uint32_t(((16 * ks) / HALF) * HALF + ((16 * ks) % HALF) / 2);
-      };
-      auto wait_st_free = [&](int b) {
-        if (st_commits[b] > st_waits[b]) {
-          ok = ok && mbar_wait(&bars.st_free[b], st_waits[b] & 1, wctx);
-          ++st_waits[b];
-        }
-      };
-      auto wait_dpt_free = [&]() {
-        if (dpt_commits > dpt_waits) {
-          ok = ok && mbar_wait(&bars.dpt_free, dpt_waits & 1, wctx);
-          ++dpt_waits;
-        }
-      };
-      auto issue_st = [&](int st, int b) {       // S^T = K Q^T
-        for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + Cfg::TM_ST + b * BQ, sdesc_sw128(sK + kb * BKV * 128 + ks * 32, 16, 1024),
-                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
-                   idesc_s, (kb | ks) != 0);
-      };
-      auto issue_dpt = [&](int st) {             // dP^T = V dO^T
-        for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_ss(tmem + Cfg::TM_DPT, sdesc_sw128(sV + kb * BKV * 128 + ks * 32, 16, 1024),
-                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
-                   idesc_s, (kb | ks) != 0);
-      };
-      for (int k = 0; ok; ++k) {
-        const int slot = k % kUnitRing;
-        ok = mbar_wait(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
-        if (!ok) break;
-        const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
-        mbar_arrive(&bars.unit_empty[slot]);
-        if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
-        const uint32_t cq = uint32_t(u.c * CB * BQ * 128);   // chunk offset in a Q / dO tile
-        const uint32_t ck = uint32_t(u.c * CB * BKV * 128);  // chunk offset in the K tile
-        ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
-        kv_ph ^= 1;
-        if (!ok) break;
-        SlotWalk w;
-        bool more = walk_first(prm, u.n, w);
-        // prologue: S^T(0), dP^T(0)
-        if (more) {
-          const int st = int(q_it & 1);
-          ok = mbar_wait(&bars.q_full[st], q_full_uses[st] & 1, wctx);
-          ++q_full_uses[st];
-          wait_st_free(0);
-          if (!ok) break;
-          tc_fence_after();
-          issue_st(st, 0);
-          mma_commit(&bars.s_full[0]);
-          wait_dpt_free();
-          if (!ok) break;
-          tc_fence_after();
-          issue_dpt(st);
-          mma_commit(&bars.dp_full);
-        }
-        for (int j = 0; more && ok; ++j) {
-          const int b = j & 1;
-          const int st = int(q_it & 1);
-          SlotWalk nx = w;
-          const bool has_next = walk_next(prm, u.n, nx);
-          const int st1 = int((q_it + 1) & 1);
-          // dV += P^T dO
-          ok = mbar_wait(&bars.p_full, p_ph, wctx);
-          p_ph ^= 1;
-          if (ok && j == 0 && acc_commits > 0)
-            ok = mbar_wait(&bars.acc_empty, (acc_commits - 1) & 1, wctx);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < BQ / 16; ++ks)
-            mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + b * BQ + p_col(ks),
-                   sdesc_sw128(sDO + st * Cfg::QT_BYTES + cq + ks * 2048, BQ * 128, 1024), idesc_kv,
-                   (j > 0) || (ks > 0));
-          mma_commit(&bars.st_free[b]);
-          ++st_commits[b];
-          // next slot's S^T into the other buffer
-          if (has_next) {
-            ok = mbar_wait(&bars.q_full[st1], q_full_uses[st1] & 1, wctx);
-            ++q_full_uses[st1];
-            wait_st_free(b ^ 1);
-            if (!ok) break;
-            tc_fence_after();
-            issue_st(st1, b ^ 1);
-            mma_commit(&bars.s_full[b ^ 1]);
-          }
-          // dK += dS^T Q ; dQ^T = K^T dS^T
-          ok = mbar_wait(&bars.ds_full, ds_ph, wctx);
-          ds_ph ^= 1;
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < BQ / 16; ++ks)
-            mma_ts(tmem + Cfg::TM_DK, tmem + Cfg::TM_DPT + p_col(ks),
-                   sdesc_sw128(sQ + st * Cfg::QT_BYTES + cq + ks * 2048, BQ * 128, 1024), idesc_kv,
-                   (j > 0) || (ks > 0));
-          mma_commit(&bars.dpt_free);
-          ++dpt_commits;
-          if (dq_commits > dq_waits) {
-            ok = mbar_wait(&bars.dq_empty, dq_waits & 1, wctx);
-            ++dq_waits;
-            if (!ok) break;
-            tc_fence_after();
-          }
-#pragma unroll
-          for (int ks = 0; ks < BKV / 16; ++ks) {
-            const uint64_t bdesc =
-                Cfg::DS_KMAJOR
-                    ? sdesc_sw128(sDS + b * Cfg::DS_BYTES + (ks >> 2) * BQ * 128 + (ks & 3) * 32, 16, 1024)
-                    : sdesc_sw128(sDS + b * Cfg::DS_BYTES + ks * 2048, BQ * 128, 1024);
-            mma_ss(tmem + Cfg::TM_DQT, sdesc_sw128(sK + ck + ks * 2048, lbo_kt, 1024), bdesc,
-                   idesc_dq, ks > 0);
-          }
-          mma_commit(&bars.dq_full);
-          ++dq_commits;
-          mma_commit(&bars.dsm_free[b]);
-          mma_commit(&bars.q_empty[st]);
-          ++q_it;
-          // next slot's dP^T once dK has consumed dS^T from the dP^T columns
-          if (has_next) {
-            wait_dpt_free();
-            if (!ok) break;
-            tc_fence_after();
-            issue_dpt(st1);
-            mma_commit(&bars.dp_full);
-          }
-          w = nx;
-          more = has_next;
-        }
-        if (!ok) break;
-        mma_commit(&bars.acc_full);
-        ++acc_commits;
-        mma_commit(&bars.kv_empty);
-      }
-      mma_commit(&bars.drain);
-      mbar_drain(&bars.drain, 0, 1000000000ull);
-    }
-    __syncwarp();
-  } else if (warp >= Cfg::WARP_DQ) {
-    // ------------------------------------------------------------ dQ warps
-    const int qw = warp - Cfg::WARP_DQ;
-    const int drow = qw * 32 + lane;           // TMEM lane = d index (within the chunk) of dQ^T
-    const uint32_t tDQ = tmem + Cfg::TM_DQT + (uint32_t(qw * 32) << 16);
-    uint32_t dq_ph = 0;
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int slot = k % kUnitRing;
-      ok = warp_wait_b(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
-      if (!ok) break;
-      const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
-      if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
-      SlotWalk w;
-      for (bool more = walk_first(prm, u.n, w); more; more = walk_next(prm, u.n, w)) {
-        ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
-        dq_ph ^= 1;
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t v[BQ / 32][32];
-#pragma unroll
-        for (int t = 0; t < BQ / 32; ++t) tmem_ld32(tDQ + t * 32, v[t]);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.dq_empty);
-        if (drow < HC) {
-          const int32_t h = u.g * prm.G + w.e;
-          const int64_t row0 = (int64_t(w.r - prm.shard_begin) * prm.B + u.b) * twoC + int64_t(w.i) * BQ;
-          // head-major accumulator [Hq][rows][d]
-          float* base = prm.dq_acc + (int64_t(h) * prm.rows + row0) * HD + u.c * HC + drow;
-          const int64_t rstride = HD;
-#pragma unroll
-          for (int t = 0; t < BQ / 32; ++t)
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              atomicAdd(base + (t * 32 + c) * rstride, __uint_as_float(v[t][c]));
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ compute warps
-    const int half = warp / 4;                 // which HALF of the slot's BQ columns
-    const int qw = warp % 4;
-    const int row = qw * 32 + lane;            // TMEM lane = key within the tile
-    const uint32_t lane_addr = uint32_t(qw * 32) << 16;
-    const float* sLse = reinterpret_cast<const float*>(smem + Cfg::SMEM_LSE);
-    const float* sDelta = reinterpret_cast<const float*>(smem + Cfg::SMEM_DELTA);
-    uint8_t* sDS = smem + Cfg::SMEM_DS;
-    uint32_t q_it = 0, q_full_uses[2] = {0, 0};
-    uint32_t s_ph[2] = {0, 0}, dp_ph = 0, acc_ph = 0;
-    uint32_t dsm_uses[2] = {0, 0};
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int slot = k % kUnitRing;
-      ok = warp_wait_b(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
-      if (!ok) break;
-      const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
-      if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, Cfg::NCHUNK);
-      const int64_t key = int64_t(u.n) * BKV + row;
-      SlotWalk w;
-      int j = 0;
-      for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w), ++j) {
-        const int b = j & 1;
-        const int st = int(q_it & 1);
-        ok = warp_wait_b(&bars.q_full[st], q_full_uses[st] & 1, wctx);
-        ++q_full_uses[st];
-        if (!ok) break;
-        // per-column statistics of this warp's 32 query rows, read from shared memory
-        const float* lse_c = sLse + st * BQ + half * HALF;
-        const float* dlt_c = sDelta + st * BQ + half * HALF;
-        // causal mask: column c holds position p0 + half*HALF + c; masked when key > it
-        const int64_t first = w.p0 + half * HALF;
-        const int nvis_lo = prm.causal ? int(key - first) : 0;   // columns c < nvis_lo are masked
-        // ---- P^T
-        ok = warp_wait_b(&bars.s_full[b], s_ph[b], wctx);
-        s_ph[b] ^= 1;
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sv[HALF];
-        tmem_ld_n<HALF>(tmem + Cfg::TM_ST + b * BQ + half * HALF + lane_addr, sv);
-        tmem_ld_wait();
-        float pf[HALF];
-        uint32_t pk[HALF / 2];
-#pragma unroll
-        for (int c = 0; c < HALF; ++c) {
-          const float x = fmaf(__uint_as_float(sv[c]), prm.scale_log2, -lse_c[c] * kLog2e);
-          pf[c] = (c < nvis_lo) ? 0.f : ex2_approx(x);
-        }
-#pragma unroll
-        for (int e = 0; e < HALF / 2; ++e) pk[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
-        tmem_st_n<HALF / 2>(tmem + Cfg::TM_ST + b * BQ + half * HALF + lane_addr, pk);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full);
-        // ---- dS^T
-        ok = warp_wait_b(&bars.dp_full, dp_ph, wctx);
-        dp_ph ^= 1;
-        if (!ok) break;
-        tc_fence_after();
-        tmem_ld_n<HALF>(tmem + Cfg::TM_DPT + half * HALF + lane_addr, sv);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < HALF / 2; ++e)
-          pk[e] = pack_bf16x2(pf[2 * e] * (__uint_as_float(sv[2 * e]) - dlt_c[2 * e]),
-                              pf[2 * e + 1] * (__uint_as_float(sv[2 * e + 1]) - dlt_c[2 * e + 1]));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.q_empty[st]);   // lse / Delta of this stage consumed
-        ++q_it;
-        tmem_st_n<HALF / 2>(tmem + Cfg::TM_DPT + half * HALF + lane_addr, pk);
-        // shared-memory copy of dS for the dQ MMA
-        if (dsm_uses[b] > 0) {
-          ok = warp_wait_b(&bars.dsm_free[b], (dsm_uses[b] - 1) & 1, wctx);
-          if (!ok) break;
-        }
-        ++dsm_uses[b];
-        uint8_t* dsb = sDS + b * Cfg::DS_BYTES;
-        if constexpr (!Cfg::DS_KMAJOR) {
-          // MN-major [key][64 q]: row = key, 16-byte chunks 4*half .. 4*half+3
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            *reinterpret_cast<uint4*>(dsb + sw128_offset(uint32_t(row), uint32_t(4 * half + m))) =
-                make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-        } else {
-          // K-major [q][keys] in 64-key blocks of BQ rows x 128 B: element (q, key) sits
-          // in block key/64, row q, 16-byte chunk ((key%64)/8) ^ (q%8), bytes 2*(key%8)
-          uint8_t* blk = dsb + (row >> 6) * (BQ * 128);
-          const uint32_t kc = uint32_t((row & 63) >> 3), kb2 = uint32_t((row & 7) * 2);
-#pragma unroll
-          for (int e = 0; e < HALF / 2; ++e) {
-            const uint32_t q0 = uint32_t(half * HALF + 2 * e);
-            *reinterpret_cast<uint16_t*>(blk + q0 * 128 + ((kc ^ (q0 & 7)) << 4) + kb2) =
-                uint16_t(pk[e] & 0xFFFFu);
-            *reinterpret_cast<uint16_t*>(blk + (q0 + 1) * 128 + ((kc ^ ((q0 + 1) & 7)) << 4) + kb2) =
-                uint16_t(pk[e] >> 16);
-          }
-        }
-        fence_proxy_async_smem();
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.ds_full);
-      }
-      if (!ok) break;
-      // ---- epilogue: dV (first group) / dK (second group) rows of this key tile
-      ok = warp_wait_b(&bars.acc_full, acc_ph, wctx);
-      acc_ph ^= 1;
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t tAcc = tmem + (half == 0 ? Cfg::TM_DV : Cfg::TM_DK) + lane_addr;
-      const float mul = half == 0 ? 1.0f : prm.scale;
-      const int64_t krow = kv_tensor_row(key, u.b, prm.S, prm.B, prm.D, prm.kv_shard_major);
-      __nv_bfloat16* dst = (half == 0 ? prm.dv : prm.dk) + (krow * prm.Hkv + u.g) * HD + u.c * HC;
-      // a key tile no query of the launch's shards sees has no MMA behind its
-      // accumulators: its dK / dV rows are zero
-      const bool empty = j == 0;
-#pragma unroll 1
-      for (int c = 0; c < HC / 32; ++c) {
-        uint32_t a[32];
-        if (!empty) {
-          tmem_ld32(tAcc + c * 32, a);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) a[e] = 0u;
-        }
-        uint32_t o16[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          o16[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * mul, __uint_as_float(a[2 * e + 1]) * mul);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          d4[v4] = make_uint4(o16[4 * v4], o16[4 * v4 + 1], o16[4 * v4 + 2], o16[4 * v4 + 3]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.acc_empty);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == Cfg::WARP_MMA) tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
 // ------------------------------------------------------------------ K3 for d <= 128
@@ -1267,12 +637,11 @@ int num_sms() {
 
 template <int HD>
 int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
-  // d <= 128: 128-row q slots (all MMAs N = 128); d = 256: 32-row slots over two d chunks
+  // 128-key tiles and 128-row q slots (every MMA N >= 128).  d <= 128: one CTA per key
+  // tile (zsa_bwd_wide_kernel); d = 256: a cluster of two CTAs per key tile
+  // (zsa_bwd_pair_kernel), since dK + dV of the tile alone fill one SM's TMEM.
   constexpr bool kWide = HD <= 128;
-  using Cfg = std::conditional_t<kWide, BwdWideCfg<HD>, BwdCfg<HD>>;
-  constexpr int kChunks = kWide ? 1 : HD / 128;    // d chunks of 128 per key tile
-  // the 128-row kernel aligns its dynamic shared memory itself (no slack needed)
-  constexpr int kSmem = kWide ? Cfg::SMEM_BYTES : Cfg::SMEM_BYTES + 1024;
+  constexpr int BQ = 128, BKV = 128;
   const int64_t twoC = a.S / a.D;
   const int64_t rows = int64_t(a.shard_count) * a.B * twoC;   // local shard-major rows
   const int sms = num_sms();
@@ -1297,7 +666,7 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hq), uint64_t(rows)};
     const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hq) * HD * 2};
-    const uint32_t box[3] = {64, 1, uint32_t(Cfg::BQ)};
+    const uint32_t box[3] = {64, 1, uint32_t(BQ)};
     if (!make_map_bf16_sw128(&mq, a.q, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
     if (!make_map_bf16_sw128(&mdo, a.dout, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
@@ -1308,11 +677,11 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
     if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
     if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
-  CUtensorMap mdq;
-  if constexpr (kWide) {
+  CUtensorMap mdq;   // the head-major fp32 dQ accumulator, [128 rows][32 d] reduce boxes
+  {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(rows), uint64_t(a.Hq)};
     const uint64_t strides[2] = {uint64_t(HD) * 4, uint64_t(rows) * HD * 4};
-    const uint32_t box[3] = {32, uint32_t(Cfg::BQ), 1};
+    const uint32_t box[3] = {32, uint32_t(BQ), 1};
     if (!make_map_f32_sw128(&mdq, a.dq_acc, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
   BwdParams p;
@@ -1324,11 +693,11 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.S = a.S;
   p.C = a.S / (2 * int64_t(a.D));
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = a.Hq / a.Hkv; p.D = a.D; p.causal = a.causal;
-  p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / Cfg::BKV) * kChunks);
-  p.n_qtiles = int32_t(twoC / Cfg::BQ);
-  p.n_chunks = kChunks;
-  p.bq = Cfg::BQ;
-  p.n_ktiles = int32_t(a.S / Cfg::BKV);
+  p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / BKV));
+  p.n_qtiles = int32_t(twoC / BQ);
+  p.n_chunks = 1;
+  p.bq = BQ;
+  p.n_ktiles = int32_t(a.S / BKV);
   p.kv_shard_major = a.kv_layout;
   p.shard_begin = a.shard_begin;
   p.shard_end = a.shard_begin + a.shard_count;
@@ -1339,24 +708,23 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
   p.inject_stall = a.inject_stall;
-  const int smem = kSmem;
-  auto kernel = [] {
-    if constexpr (kWide) return zsa_bwd_wide_kernel<HD>;
-    else return zsa_bwd_kernel<HD>;
-  }();
-  {
-    const int e = ensure_smem_attr(reinterpret_cast<const void*>(kernel), smem);
-    if (e != int(cudaSuccess)) return e;
+  cudaError_t e = cudaSuccess;
+  if constexpr (kWide) {
+    using Cfg = BwdWideCfg<HD>;
+    const int smem = Cfg::SMEM_BYTES;   // the kernel aligns its dynamic shared memory itself
+    {
+      const int err = ensure_smem_attr(reinterpret_cast<const void*>(zsa_bwd_wide_kernel<HD>), smem);
+      if (err != int(cudaSuccess)) return err;
+    }
+    const int grid = p.n_units < sms ? p.n_units : sms;
+    const TraceEvents tr = trace_events(2);
+    if (tr.begin) cudaEventRecord(tr.begin, stream);
+    zsa_bwd_wide_kernel<HD><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
+    e = cudaGetLastError();
+    if (tr.end) cudaEventRecord(tr.end, stream);
+  } else {
+    e = cudaError_t(launch_pair_main(mq, mk, mv, mdo, mdq, p, stream));
   }
-  const int grid = p.n_units < sms ? p.n_units : sms;
-  const TraceEvents tr = trace_events(2);
-  if (tr.begin) cudaEventRecord(tr.begin, stream);
-  if constexpr (kWide)
-    kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
-  else
-    kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, mdo, p);
-  cudaError_t e = cudaGetLastError();
-  if (tr.end) cudaEventRecord(tr.end, stream);
   if (e != cudaSuccess) return int(e);
   // K4
   {
