@@ -407,10 +407,18 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="zsa", choices=("zsa", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="run the configuration's heads, d and D at this sequence length "
+                         "(profiling captures of a smaller case); 0 = the configuration's S")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    c = CONFIGS[args.config]
+    c = dict(CONFIGS[args.config])
+    if args.seq:
+        if args.seq % (2 * c["D"] * 128):
+            ap.error(f"--seq must be a multiple of 2*D*128 = {2 * c['D'] * 128}")
+        c["desc"] = c["desc"].replace(f"S={c['S']}", f"S={args.seq}") + " (reduced S)"
+        c["S"] = args.seq
     _, world, _ = dist_env()
     if world != args.gpus and not (world == 1 and args.gpus == 1):
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)

@@ -191,6 +191,32 @@ ZSA_API int zsa_attn_merge(const zsa_problem* problem, int32_t n_parts, const vo
                            const float* const* lse_parts, void* o, float* lse,
                            void* cuda_stream);
 
+/* One run of output columns of a TSP projection step (zsa_tsp_project). */
+typedef struct {
+  void* out;                 /* device: element (0, 0) of this run's output */
+  int64_t ld;                /* row stride of out, in elements (a multiple of 8) */
+  int32_t cols;              /* columns of W routed here (a multiple of 32) */
+  int32_t fp32_accumulate;   /* 0: out is bf16 and overwritten; 1: out is fp32, out += */
+} zsa_proj_segment;
+
+#define ZSA_PROJ_MAX_SEGMENTS 8
+
+/* One step of the TSP attention-layer weight schedule on one rank ("Folding Tensor and
+ * Sequence Parallelism" summary, section 2, attention layer: each rank holds 1/D of the
+ * tokens and one packed shard of W_Q/W_K/W_V/W_O; step s broadcasts rank s's shard and
+ * every rank projects its own tokens with it):
+ *   Y = X W,   X [T][K] bf16 (row stride ldx), W [K][N] bf16 (row stride ldw),
+ * with Y's columns routed, in order, to segs[0], segs[1], ... (segs[i].cols each, summing
+ * to N): e.g. the Q, K and V columns of the shard's heads written into the rank's Q, K
+ * and V (bf16), or the output projection's partial added into an fp32 accumulator.
+ * T, N multiples of 128; K a multiple of 64; ldx, ldw multiples of 8; x, w and every
+ * out 16-byte aligned.  `status_ws` is a 256-byte device workspace whose status word
+ * zsa_device_status reads (a bounded wait that gave up).  Asynchronous on cuda_stream.
+ * fp32 tensor-core accumulation; bf16 outputs rounded to nearest even. */
+ZSA_API int zsa_tsp_project(int64_t T, int64_t K, int64_t N, const void* x, int64_t ldx,
+                            const void* w, int64_t ldw, const zsa_proj_segment* segs,
+                            int32_t n_segs, void* status_ws, void* cuda_stream);
+
 /* Size of the fixed device scratch behind zsa_attn_bwd_noalloc (64 MiB per device). */
 #define ZSA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
@@ -245,10 +271,11 @@ ZSA_API int zsa_debug_inject_stall(int enable);
  * launch stream immediately before / after the kernel, so the caller can time that
  * kernel alone with cudaEventElapsedTime.  which: ZSA_TRACE_FWD (forward kernel),
  * ZSA_TRACE_BWD_PRE (Delta preprocess), ZSA_TRACE_BWD_MAIN (backward main kernel),
- * ZSA_TRACE_BWD_DQ (dQ conversion), ZSA_TRACE_MERGE (partial-result merge).  Pass NULL events to stop tracing that kernel. */
+ * ZSA_TRACE_BWD_DQ (dQ conversion), ZSA_TRACE_MERGE (partial-result merge),
+ * ZSA_TRACE_PROJ (TSP projection GEMM).  Pass NULL events to stop tracing that kernel. */
 enum {
   ZSA_TRACE_FWD = 0, ZSA_TRACE_BWD_PRE = 1, ZSA_TRACE_BWD_MAIN = 2, ZSA_TRACE_BWD_DQ = 3,
-  ZSA_TRACE_MERGE = 4
+  ZSA_TRACE_MERGE = 4, ZSA_TRACE_PROJ = 5
 };
 ZSA_API int zsa_trace_events(int which, void* begin_event, void* end_event);
 

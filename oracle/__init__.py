@@ -230,3 +230,11 @@ def attn_merge(o_parts, lse_parts):
     if rc != 0:
         raise ValueError("oracle_attn_merge: invalid arguments")
     return o, np.ascontiguousarray(lse_flat.transpose(0, 1, 3, 2))
+
+
+def project(x, w):
+    """One local projection of the TSP attention-layer schedule, Y = X W, in fp64 from the
+    (bf16) input values.  "Folding Tensor and Sequence Parallelism" summary, section 2,
+    attention layer: every broadcast step multiplies the rank's tokens by the shard of
+    the packed attention weights it received.  The matmul is a library step."""
+    return _f64(x) @ _f64(w)

@@ -35,10 +35,12 @@ ZSA_KV_SHARD_MAJOR = 1
 
 EXPORTED = ("zsa_partition", "zsa_workspace_bytes", "zsa_attn_fwd", "zsa_attn_bwd",
             "zsa_device_status", "zsa_set_wait_limit_ns", "zsa_debug_inject_stall",
-            "zsa_trace_events", "zsa_attn_merge", "zsa_attn_bwd_noalloc",
+            "zsa_trace_events", "zsa_attn_merge", "zsa_tsp_project", "zsa_attn_bwd_noalloc",
             "zsa_noalloc_status", "zsa_status_string")
 ZSA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
-ZSA_TRACE_FWD, ZSA_TRACE_BWD_PRE, ZSA_TRACE_BWD_MAIN, ZSA_TRACE_BWD_DQ, ZSA_TRACE_MERGE = range(5)
+(ZSA_TRACE_FWD, ZSA_TRACE_BWD_PRE, ZSA_TRACE_BWD_MAIN, ZSA_TRACE_BWD_DQ, ZSA_TRACE_MERGE,
+ ZSA_TRACE_PROJ) = range(6)
+ZSA_PROJ_MAX_SEGMENTS = 8
 ZSA_MERGE_MAX_PARTS = 32
 
 
@@ -57,6 +59,11 @@ class zsa_tiling(ctypes.Structure):
 class zsa_work(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("shard", "b", "kv_head", "q_tile0", "q_head0",
                                               "q_tile1", "q_head1", "k_tile_end0", "k_tile_end1")]
+
+
+class zsa_proj_segment(ctypes.Structure):
+    _fields_ = [("out", ctypes.c_void_p), ("ld", ctypes.c_int64), ("cols", ctypes.c_int32),
+                ("fp32_accumulate", ctypes.c_int32)]
 
 
 class ZsaError(RuntimeError):
@@ -88,6 +95,8 @@ def lib():
         L.zsa_debug_inject_stall.argtypes = [ctypes.c_int]
         L.zsa_trace_events.argtypes = [ctypes.c_int, vp, vp]
         L.zsa_attn_merge.argtypes = [P(zsa_problem), ctypes.c_int32, vp, vp, vp, vp, vp]
+        i64 = ctypes.c_int64
+        L.zsa_tsp_project.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, ctypes.c_int32, vp, vp]
         L.zsa_attn_bwd_noalloc.argtypes = [P(zsa_problem)] + [vp] * 10
         L.zsa_noalloc_status.argtypes = [vp]
         L.zsa_status_string.argtypes = [ctypes.c_int]
@@ -195,6 +204,23 @@ def zsa_attn_merge(problem, o_parts, lse_parts, o, lse, stream=None):
     _check(lib().zsa_attn_merge(ctypes.byref(problem), n, ctypes.cast(op, ctypes.c_void_p),
                                 ctypes.cast(lp, ctypes.c_void_p), _ptr(o), _ptr(lse),
                                 _stream(stream)), "zsa_attn_merge")
+
+
+def zsa_tsp_project(x, w, segments, status_ws, T=None, K=None, N=None, ldx=None, ldw=None,
+                    stream=None):
+    """Y = X W for one TSP step, Y's columns routed to `segments`: a list of
+    (out, ld, cols, fp32_accumulate), out a tensor / device pointer."""
+    if T is None:
+        T, K = x.shape[0], x.shape[1]
+    if N is None:
+        N = w.shape[1]
+    ldx = x.stride(0) if ldx is None else ldx
+    ldw = w.stride(0) if ldw is None else ldw
+    segs = (zsa_proj_segment * len(segments))(
+        *[zsa_proj_segment(_ptr(o), int(ld), int(c), int(bool(acc))) for o, ld, c, acc in segments])
+    _check(lib().zsa_tsp_project(int(T), int(K), int(N), _ptr(x), int(ldx), _ptr(w), int(ldw),
+                                 ctypes.cast(segs, ctypes.c_void_p), len(segments),
+                                 _ptr(status_ws), _stream(stream)), "zsa_tsp_project")
 
 
 def zsa_attn_bwd_noalloc(problem, q, k, v, o, lse, dout, dq, dk, dv, stream=None):

@@ -27,7 +27,7 @@ using zsa::Schedule;
 constexpr size_t kStatusBytes = 256;
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_inject_stall{0};
-constexpr int kTraceKernels = 5;
+constexpr int kTraceKernels = 6;
 std::atomic<void*> g_trace_begin[kTraceKernels];
 std::atomic<void*> g_trace_end[kTraceKernels];
 
@@ -367,6 +367,46 @@ int zsa_attn_merge(const zsa_problem* problem, int32_t n_parts, const void* cons
   a.Hq = problem->Hq; a.d = problem->d; a.D = problem->D; a.n = n_parts;
   if (zsa::launch_merge(a, static_cast<cudaStream_t>(cuda_stream)) != int(cudaSuccess))
     return ZSA_ERR_CUDA;
+  return ZSA_OK;
+}
+
+int zsa_tsp_project(int64_t T, int64_t K, int64_t N, const void* x, int64_t ldx, const void* w,
+                    int64_t ldw, const zsa_proj_segment* segs, int32_t n_segs, void* status_ws,
+                    void* cuda_stream) {
+  if (!x || !w || !segs || !status_ws) return ZSA_ERR_INVALID;
+  if (T <= 0 || K <= 0 || N <= 0 || ldx < K || ldw < N) return ZSA_ERR_INVALID;
+  if (T % 128 || N % 128 || K % 64) return ZSA_ERR_SHAPE;
+  if (ldx % 8 || ldw % 8 || !aligned16(x) || !aligned16(w) ||
+      (reinterpret_cast<uintptr_t>(status_ws) & 255))
+    return ZSA_ERR_INVALID;
+  if (T >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+    return ZSA_ERR_SHAPE;
+  if (n_segs < 1 || n_segs > ZSA_PROJ_MAX_SEGMENTS) return ZSA_ERR_INVALID;
+  zsa::ProjArgs a;
+  int64_t col = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    const zsa_proj_segment& g = segs[i];
+    if (!g.out || g.cols <= 0 || g.cols % 32 || g.ld % 8 || !aligned16(g.out) ||
+        (g.fp32_accumulate != 0 && g.fp32_accumulate != 1) || g.ld < g.cols)
+      return ZSA_ERR_INVALID;
+    a.segs[i].out = g.out;
+    a.segs[i].ld = g.ld;
+    a.segs[i].col_begin = col;
+    a.segs[i].col_end = col + g.cols;
+    a.segs[i].fp32_accumulate = g.fp32_accumulate;
+    col += g.cols;
+  }
+  if (col != N) return ZSA_ERR_INVALID;
+  int rc = check_sm100();
+  if (rc) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaMemsetAsync(status_ws, 0, kStatusBytes, stream) != cudaSuccess) return ZSA_ERR_CUDA;
+  a.x = x; a.w = w;
+  a.T = T; a.N = N; a.K = K; a.ldx = ldx; a.ldw = ldw;
+  a.n_segs = n_segs;
+  a.status = static_cast<int*>(status_ws);
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  if (zsa::launch_proj_gemm(a, stream) != int(cudaSuccess)) return ZSA_ERR_CUDA;
   return ZSA_OK;
 }
 

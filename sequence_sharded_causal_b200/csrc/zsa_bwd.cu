@@ -256,13 +256,13 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
-        for (int hb = 0; hb < BKV / 64; ++hb) {
-          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * 64, u.b, prm.S, prm.B, prm.D,
+        for (int hb = 0; hb < BKV / prm.kv_box; ++hb) {
+          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * prm.kv_box, u.b, prm.S, prm.B, prm.D,
                                              prm.kv_shard_major);
           for (int kb = 0; kb < KB; ++kb) {
-            tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128 + hb * 64 * 128, &map_k, &bars.kv_full,
+            tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128 + hb * prm.kv_box * 128, &map_k, &bars.kv_full,
                         kb * 64, u.g, krow);
-            tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128 + hb * 64 * 128, &map_v, &bars.kv_full,
+            tma_load_3d(smem + Cfg::SMEM_V + kb * BKV * 128 + hb * prm.kv_box * 128, &map_v, &bars.kv_full,
                         kb * 64, u.g, krow);
           }
         }
@@ -673,7 +673,8 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), uint64_t(a.B * a.S)};
     const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hkv) * HD * 2};
-    const uint32_t box[3] = {64, 1, 64};   // 64-key boxes: one zigzag chunk each
+    // a box never straddles a zigzag chunk: its rows are contiguous in both layouts
+    const uint32_t box[3] = {64, 1, uint32_t((a.S / (2 * int64_t(a.D))) % BKV == 0 ? BKV : 64)};
     if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
     if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
@@ -699,6 +700,7 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.bq = BQ;
   p.n_ktiles = int32_t(a.S / BKV);
   p.kv_shard_major = a.kv_layout;
+  p.kv_box = (a.S / (2 * int64_t(a.D))) % BKV == 0 ? BKV : 64;
   p.shard_begin = a.shard_begin;
   p.shard_end = a.shard_begin + a.shard_count;
   p.rows = rows;

@@ -24,6 +24,7 @@ struct BwdParams {
   int32_t n_chunks, bq;       // d chunks per key tile, query rows per slot
   int32_t n_ktiles;           // S / 128
   int32_t kv_shard_major;     // K/V/dK/dV rows in the shard-major zigzag order
+  int32_t kv_box;             // rows per K / V TMA box (128, or 64 when C % 128 != 0)
   int32_t shard_begin, shard_end;   // the launch computes the queries of these shards
   int64_t rows;               // local Q-layout rows: (shard_end - shard_begin) * B * 2C
   float scale, scale_log2;

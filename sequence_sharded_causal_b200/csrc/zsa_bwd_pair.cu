@@ -192,11 +192,11 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         if (t_fills > 0) ok = mbar_wait(&bars.t_empty, (t_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.t_full, Cfg::TILE_BYTES);
-        for (int hb = 0; hb < BKV / 64; ++hb) {
-          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * 64, u.b, prm.S, prm.B, prm.D,
+        for (int hb = 0; hb < BKV / prm.kv_box; ++hb) {
+          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * prm.kv_box, u.b, prm.S, prm.B, prm.D,
                                              prm.kv_shard_major);
           for (int kb = 0; kb < KB; ++kb)
-            tma_load_3d(smem + Cfg::SMEM_T + kb * BKV * 128 + hb * 64 * 128,
+            tma_load_3d(smem + Cfg::SMEM_T + kb * BKV * 128 + hb * prm.kv_box * 128,
                         rank == 0 ? &map_k : &map_v, &bars.t_full, kb * 64, u.g, krow);
         }
         ++t_fills;

@@ -75,6 +75,8 @@ struct FwdParams {
   int32_t B, Hq, Hkv, D, causal;
   int32_t kv_shard_major;  // K/V rows in the shard-major zigzag order instead of position order
   int32_t shard_begin;     // first shard this launch computes (Q-layout rows are local)
+  int32_t kv_box;          // rows per K / V TMA box: BK when a key tile never straddles a
+                           // zigzag chunk (C % BK == 0), else 64 (C is a multiple of 64)
   float scale_log2;
   int* status;
   int* counter;       // next unclaimed unit (zeroed before every launch)
@@ -223,11 +225,11 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.k_full[st], Cfg::KV_BYTES);
-            for (int hb = 0; hb < BK / 64; ++hb) {
-              const int32_t krow = kv_tensor_row(int64_t(n) * BK + hb * 64, u.b, prm.S, prm.B,
+            for (int hb = 0; hb < BK / prm.kv_box; ++hb) {
+              const int32_t krow = kv_tensor_row(int64_t(n) * BK + hb * prm.kv_box, u.b, prm.S, prm.B,
                                                  prm.D, prm.kv_shard_major);
               for (int kb = 0; kb < KB; ++kb)
-                tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
+                tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128 + hb * prm.kv_box * 128,
                             &map_k, &bars.k_full[st], kb * 64, u.g, krow);
             }
             ++k_fills[st];
@@ -239,11 +241,11 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.v_full[st], Cfg::KV_BYTES);
-            for (int hb = 0; hb < BK / 64; ++hb) {
-              const int32_t vrow = kv_tensor_row(int64_t(n - 1) * BK + hb * 64, u.b, prm.S, prm.B,
+            for (int hb = 0; hb < BK / prm.kv_box; ++hb) {
+              const int32_t vrow = kv_tensor_row(int64_t(n - 1) * BK + hb * prm.kv_box, u.b, prm.S, prm.B,
                                                  prm.D, prm.kv_shard_major);
               for (int kb = 0; kb < KB; ++kb)
-                tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
+                tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128 + hb * prm.kv_box * 128,
                             &map_v, &bars.v_full[st], kb * 64, u.g, vrow);
             }
             ++v_fills[st];
@@ -537,6 +539,7 @@ template <int HD>
 int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   using Cfg = FwdCfg<HD>;
   const int64_t rows = int64_t(a.shard_count) * a.B * (a.S / a.D);  // local shard-major rows
+  const int32_t kv_box = (a.S / (2 * int64_t(a.D))) % Cfg::BK == 0 ? Cfg::BK : 64;
   CUtensorMap mq, mk, mv;
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hq), uint64_t(rows)};
@@ -547,7 +550,9 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), uint64_t(a.B * a.S)};
     const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hkv) * HD * 2};
-    const uint32_t box[3] = {64, 1, 64};   // 64-key boxes: one zigzag chunk each
+    // a box never straddles a zigzag chunk: the K/V rows it covers are contiguous in
+    // both layouts
+    const uint32_t box[3] = {64, 1, uint32_t(kv_box)};
     if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
     if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
@@ -561,6 +566,7 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.D = a.D; p.causal = a.causal;
   p.kv_shard_major = a.kv_layout;
   p.shard_begin = a.shard_begin;
+  p.kv_box = kv_box;
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
   p.status = a.status;
   p.counter = a.status + 32;

@@ -60,6 +60,25 @@ struct MergeArgs {
   int32_t Hq, d, D, n;
 };
 
+// One TSP step's local projection Y = X W (zsa_gemm.cu): X [T][K] (row stride ldx),
+// W [K][N] (row stride ldw), columns of Y routed by segments.
+constexpr int kProjMaxSegs = 8;
+struct ProjSegment {
+  void* out;               // element (0, 0) of the segment's output
+  int64_t ld;              // its row stride (elements)
+  int64_t col_begin, col_end;   // the columns of W it receives
+  int32_t fp32_accumulate; // 0: bf16 output, overwritten; 1: fp32 output, +=
+};
+struct ProjArgs {
+  const void* x;
+  const void* w;
+  int64_t T, N, K, ldx, ldw;
+  int32_t n_segs;
+  ProjSegment segs[kProjMaxSegs];
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
 // Tiling the forward kernel is built for, per head dim.
 inline void fwd_tiling(int d, int32_t* bq, int32_t* bk, int32_t* slots) {
   *bq = 128;
@@ -71,7 +90,8 @@ inline void fwd_tiling(int d, int32_t* bq, int32_t* bk, int32_t* slots) {
 struct TraceEvents {
   cudaEvent_t begin, end;
 };
-TraceEvents trace_events(int which);  // 0 fwd, 1 bwd pre, 2 bwd main, 3 dQ convert, 4 merge
+TraceEvents trace_events(int which);  // 0 fwd, 1 bwd pre, 2 bwd main, 3 dQ convert, 4 merge,
+                                      // 5 projection GEMM
 
 // Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once
 // per (kernel, device): cudaFuncSetAttribute applies to the device current at the time
@@ -87,5 +107,6 @@ int inject_stall();
 int launch_fwd(const FwdArgs& a, cudaStream_t stream);
 int launch_bwd(const BwdArgs& a, cudaStream_t stream);
 int launch_merge(const MergeArgs& a, cudaStream_t stream);
+int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream);
 
 }  // namespace zsa

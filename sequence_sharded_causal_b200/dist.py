@@ -114,3 +114,94 @@ class ShardedAttention:
     def status(self):
         """Device status of both workspaces (synchronises): ZSA_OK or ZSA_ERR_TIMEOUT."""
         return zsa.zsa_device_status(self.ws_f) or zsa.zsa_device_status(self.ws_b)
+
+
+# ---------------------------------------------------------------- TSP weight schedule
+#
+# "Folding Tensor and Sequence Parallelism" (summary page, section 2, attention layer):
+# besides 1/D of the tokens, rank r holds one packed shard of the attention weights --
+# the Q, K and V columns of its head group, and the rows of W_O for that group -- and the
+# layer's projections iterate over the shards: at step s rank s broadcasts its shard and
+# every rank projects its own tokens with it.  After the D steps each rank holds Q, K, V
+# of all heads for its tokens (Q in the shard-major layout the attention kernels read,
+# K / V as the rank's own rows for the all-gather), and the output projection's partials,
+# one per step, summed.
+#
+# The broadcast of step s+1 is posted before the GEMM of step s is enqueued, so NCCL moves
+# the next shard while the tensor cores work on the current one (double-buffered).
+
+def qkv_columns(Hq, Hkv, d, D):
+    """Columns of W_Q, W_K, W_V in each of the D packed shards: (nq, nk, nv)."""
+    if (Hq * d) % D or (Hkv * d) % D:
+        raise ValueError("the Q and K/V projection widths must split into D shards")
+    return Hq * d // D, Hkv * d // D, Hkv * d // D
+
+
+def pack_qkv_shard(wq, wk, wv, s, D):
+    """Rank s's packed shard [hidden][nq + nk + nv] of W_Q [hidden][Hq*d], W_K, W_V."""
+    nq, nk = wq.shape[1] // D, wk.shape[1] // D
+    return torch.cat([wq[:, s * nq:(s + 1) * nq], wk[:, s * nk:(s + 1) * nk],
+                      wv[:, s * nk:(s + 1) * nk]], dim=1).contiguous()
+
+
+def wo_shard(wo, s, D):
+    """Rank s's rows of W_O [Hq*d][hidden]: the inputs of its head group."""
+    nq = wo.shape[0] // D
+    return wo[s * nq:(s + 1) * nq].contiguous()
+
+
+def _broadcast_steps(w_local, group, step_fn):
+    """Run step_fn(s, w_s) for s = 0..world-1, W_s arriving by broadcast from rank s;
+    the broadcast of s+1 overlaps step s."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    bufs = [torch.empty_like(w_local), torch.empty_like(w_local)]
+
+    def post(s):
+        b = w_local if s == rank else bufs[s % 2]
+        src = dist.get_global_rank(group, s) if group is not None else s
+        return b, dist.broadcast(b, src=src, group=group, async_op=True)
+
+    cur = post(0)
+    for s in range(world):
+        nxt = post(s + 1) if s + 1 < world else None
+        b, work = cur
+        work.wait()
+        step_fn(s, b)
+        cur = nxt
+
+
+def tsp_qkv_projection(x, w_local, q, k, v, Hq, Hkv, d, group=None, project=None,
+                       status_ws=None, stream=None):
+    """Q, K, V of the rank's tokens x [T][hidden] from the packed shards (this rank's is
+    w_local [hidden][nq + nk + nv]).  q [T][Hq*d], k / v [T][Hkv*d] (bf16) are written."""
+    import torch.distributed as dist
+    D = dist.get_world_size(group)
+    nq, nk, nv = qkv_columns(Hq, Hkv, d, D)
+    if project is None:
+        def project(s, w_s):
+            zsa.zsa_tsp_project(x, w_s, [(q[:, s * nq:], Hq * d, nq, 0),
+                                         (k[:, s * nk:], Hkv * d, nk, 0),
+                                         (v[:, s * nv:], Hkv * d, nv, 0)], status_ws,
+                                stream=stream)
+    _broadcast_steps(w_local, group, project)
+    return q, k, v
+
+
+def tsp_out_projection(o, wo_local, y32, Hq, d, group=None, project=None, status_ws=None,
+                       stream=None):
+    """y32 [T][hidden] (fp32, zeroed here) = O W_O for the rank's tokens, o [T][Hq*d],
+    summed over the steps' partials O[:, head group s] W_O[s] (this rank's rows:
+    wo_local [nq][hidden])."""
+    import torch.distributed as dist
+    D = dist.get_world_size(group)
+    nq = Hq * d // D
+    y32.zero_()
+    if project is None:
+        def project(s, w_s):
+            zsa.zsa_tsp_project(o[:, s * nq:], w_s, [(y32, y32.stride(0), y32.shape[1], 1)],
+                                status_ws, T=o.shape[0], K=nq, N=y32.shape[1],
+                                ldx=o.stride(0), stream=stream)
+    _broadcast_steps(wo_local, group, project)
+    return y32
