@@ -399,6 +399,114 @@ def run_zsa(args, c, name):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ NEXT-row components
+MODEL_HIDDEN = {"tiny": 128, "7b_mha": 4096, "8b_gqa": 4096, "wide_gqa": 5120, "long": 4096}
+
+
+def _time_events(fn, steps, warmup, dev):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / steps
+
+
+def run_component(args, c, name):
+    """One JSON line for a NEXT-row kernel on one GPU, at the configuration's sizes.
+
+    merge: one ring step's running merge, (O, lse) <- merge((O, lse), (O_s, lse_s)) in
+      place over the whole Q layout (HBM-bound: reads 2 x (2d + 4) and writes 2d + 4 bytes
+      per (row, head)); partials are seeded N(0, 1) values with lse ~ N(0, 1).
+    tsp_projection: one rank's D projection steps of the TSP attention layer (QKV from
+      the packed shards, then the output projection's fp32 partials), the rank's tokens
+      T = B*S/D, hidden = the model's width; the broadcast is local on one GPU.
+    """
+    import torch
+    import sequence_sharded_causal_b200 as zsa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, S, Hq, Hkv, d, D = (c[k] for k in ("B", "S", "Hq", "Hkv", "d", "D"))
+    peak, peak_sus, hbm, peak_src = load_peaks()
+    g = torch.Generator(device=dev).manual_seed(c["seed"])
+    if args.component == "merge":
+        problem = zsa.make_problem(B, S, Hq, Hkv, d, D)
+        shp, lshp = (D, B, S // D, Hq, d), (D, B, Hq, S // D)
+        o = torch.randn(shp, generator=g, device=dev).to(torch.bfloat16)
+        o_s = torch.randn(shp, generator=g, device=dev).to(torch.bfloat16)
+        lse = torch.randn(lshp, generator=g, device=dev)
+        lse_s = torch.randn(lshp, generator=g, device=dev)
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+        def step():
+            zsa.zsa_attn_merge(problem, [o, o_s], [lse, lse_s], o, lse)
+        zsa.zsa_trace_events(zsa.ZSA_TRACE_MERGE, ev[0], ev[1])
+        ms = _time_events(step, args.steps, args.warmup, dev)
+        kms = ev[0].elapsed_time(ev[1])
+        zsa.zsa_trace_events(zsa.ZSA_TRACE_MERGE, None, None)
+        pairs = B * S * Hq
+        nbytes = pairs * (3 * (2 * d + 4))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        line = {"metric": "ring-attention (O, lse) merge GB/s at 1 B200", "value": gbs,
+                "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16 O / fp32 lse", "data": "synthetic",
+                "config": {"workload": c["desc"] + ", running merge of 2 partials in place"},
+                "roofline": {"kernel": "zsa_merge_kernel", "bound": "hbm", "achieved": gbs,
+                             "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                             "peak_source": f"{peak_src} copy bandwidth", "traffic": None,
+                             "last_launch_ms": kms},
+                "gpu_launches": args.steps}
+    else:
+        from sequence_sharded_causal_b200 import dist as zdist
+        hidden = MODEL_HIDDEN[name]
+        T = B * S // D
+        nq, nk, nv = zdist.qkv_columns(Hq, Hkv, d, D)
+        bf = torch.bfloat16
+        x = (torch.randn(T, hidden, generator=g, device=dev)).to(bf)
+        o = (torch.randn(T, Hq * d, generator=g, device=dev)).to(bf)
+        shards = [(torch.randn(hidden, nq + nk + nv, generator=g, device=dev) * 0.02).to(bf)
+                  for _ in range(D)]
+        wo = [(torch.randn(nq, hidden, generator=g, device=dev) * 0.02).to(bf) for _ in range(D)]
+        q = torch.empty(T, Hq * d, dtype=bf, device=dev)
+        k = torch.empty(T, Hkv * d, dtype=bf, device=dev)
+        v = torch.empty_like(k)
+        y32 = torch.empty(T, hidden, dtype=torch.float32, device=dev)
+        ws = torch.empty(256, dtype=torch.uint8, device=dev)
+
+        def step():
+            for s_ in range(D):
+                zsa.zsa_tsp_project(x, shards[s_], [(q[:, s_ * nq:], Hq * d, nq, 0),
+                                                    (k[:, s_ * nk:], Hkv * d, nk, 0),
+                                                    (v[:, s_ * nv:], Hkv * d, nv, 0)], ws)
+            y32.zero_()
+            for s_ in range(D):
+                zsa.zsa_tsp_project(o[:, s_ * nq:], wo[s_], [(y32, hidden, hidden, 1)], ws,
+                                    T=T, K=nq, N=hidden, ldx=Hq * d)
+        ms = _time_events(step, args.steps, args.warmup, dev)
+        if zsa.zsa_device_status(ws) != zsa.ZSA_OK:
+            raise RuntimeError("projection GEMM reported a timeout")
+        flops = 2.0 * T * hidden * (nq + nk + nv) * D + 2.0 * T * (Hq * d) * hidden
+        tf = flops / (ms * 1e-3) / 1e12
+        line = {"metric": "TSP attention-layer projections (one rank, D steps) TFLOP/s at 1 B200",
+                "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"{c['desc']}: T={T} tokens per rank, hidden={hidden}, "
+                                       f"{D} QKV steps (N={nq + nk + nv}) + {D} output steps "
+                                       f"(K={nq}, fp32 accumulate)"},
+                "roofline": {"kernel": "zsa_proj_gemm_kernel", "bound": "tensor", "achieved": tf,
+                             "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                             "peak_source": f"{peak_src} bf16 burst", "traffic": None},
+                "gpu_launches": 2 * D * args.steps}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -407,6 +515,10 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="zsa", choices=("zsa", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--component", default="attention",
+                    choices=("attention", "merge", "tsp_projection"),
+                    help="attention: the hot path (default); merge / tsp_projection: the "
+                         "ring-attention merge or the TSP projection schedule on one GPU")
     ap.add_argument("--seq", type=int, default=0,
                     help="run the configuration's heads, d and D at this sequence length "
                          "(profiling captures of a smaller case); 0 = the configuration's S")
@@ -424,6 +536,8 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, c, args.config)
+    elif args.component != "attention":
+        run_component(args, c, args.config)
     else:
         run_zsa(args, c, args.config)
 

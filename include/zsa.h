@@ -209,7 +209,7 @@ typedef struct {
  * with Y's columns routed, in order, to segs[0], segs[1], ... (segs[i].cols each, summing
  * to N): e.g. the Q, K and V columns of the shard's heads written into the rank's Q, K
  * and V (bf16), or the output projection's partial added into an fp32 accumulator.
- * T, N multiples of 128; K a multiple of 64; ldx, ldw multiples of 8; x, w and every
+ * N a multiple of 32, K a multiple of 8 (any T); ldx, ldw multiples of 8; x, w and every
  * out 16-byte aligned.  `status_ws` is a 256-byte device workspace whose status word
  * zsa_device_status reads (a bounded wait that gave up).  Asynchronous on cuda_stream.
  * fp32 tensor-core accumulation; bf16 outputs rounded to nearest even. */

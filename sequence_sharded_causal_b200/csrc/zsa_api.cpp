@@ -375,7 +375,7 @@ int zsa_tsp_project(int64_t T, int64_t K, int64_t N, const void* x, int64_t ldx,
                     void* cuda_stream) {
   if (!x || !w || !segs || !status_ws) return ZSA_ERR_INVALID;
   if (T <= 0 || K <= 0 || N <= 0 || ldx < K || ldw < N) return ZSA_ERR_INVALID;
-  if (T % 128 || N % 128 || K % 64) return ZSA_ERR_SHAPE;
+  if (N % 32 || K % 8) return ZSA_ERR_SHAPE;
   if (ldx % 8 || ldw % 8 || !aligned16(x) || !aligned16(w) ||
       (reinterpret_cast<uintptr_t>(status_ws) & 255))
     return ZSA_ERR_INVALID;

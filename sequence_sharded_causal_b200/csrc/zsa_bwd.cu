@@ -637,11 +637,12 @@ int num_sms() {
 
 template <int HD>
 int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
-  // 128-key tiles and 128-row q slots (every MMA N >= 128).  d <= 128: one CTA per key
-  // tile (zsa_bwd_wide_kernel); d = 256: a cluster of two CTAs per key tile
-  // (zsa_bwd_pair_kernel), since dK + dV of the tile alone fill one SM's TMEM.
+  // 128-key tiles.  d <= 128: one CTA per key tile with 128-row q slots, every MMA
+  // N = 128 (zsa_bwd_wide_kernel); d = 256: a cluster of two CTAs per key tile with
+  // 64-row q slots (zsa_bwd_pair_kernel), since dK + dV of the tile alone fill one SM's
+  // TMEM.
   constexpr bool kWide = HD <= 128;
-  constexpr int BQ = 128, BKV = 128;
+  constexpr int BQ = kWide ? 128 : 64, BKV = 128;
   const int64_t twoC = a.S / a.D;
   const int64_t rows = int64_t(a.shard_count) * a.B * twoC;   // local shard-major rows
   const int sms = num_sms();

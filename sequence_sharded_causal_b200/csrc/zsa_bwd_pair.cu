@@ -2,26 +2,29 @@
 //
 // At d = 256 the fp32 dK and dV of a 128-key tile fill 512 TMEM columns, all of one
 // SM's TMEM.  This kernel splits the work of a key tile (b, kv head g, tile n) between
-// the two CTAs of a cluster by role, so that no product is computed twice and every MMA
-// has N >= 128:
+// the two CTAs of a cluster by role, so that no product is computed twice:
 //
 //   CTA 0 ("K side"): K tile resident, Q slots streamed; S^T = K Q^T, P^T = exp(scale S^T
 //     - lse) -> sent to CTA 1; dK += dS^T Q, dQ^T = K^T dS^T (two 128-row d halves).
-//     TMEM: dK (256) | ST (128) | XT (128).
+//     TMEM: dK (256) | ST x2 (64 each) | XT (dQ^T, 2 x 64).
 //   CTA 1 ("V side"): V tile resident, dO slots streamed; dP^T = V dO^T; on receiving
 //     P^T, dS^T = P^T (dP^T - Delta) -> sent to CTA 0; dV += P^T dO.
-//     TMEM: dV (256) | DT (128).
+//     TMEM: dV (256) | DT x2 (64 each).
 //
-// P^T and dS^T (bf16, 128 keys x 128 q rows, 32 KB each) cross between the CTAs through
+// q slots are 64 rows: with K (or V) resident (64 KB) that leaves room for a 3-stage
+// Q (dO) ring, double-buffered exchange buffers and a dedicated dQ staging buffer, so
+// the next slots' loads, products and exchanges overlap the current slot's.  S^T, dP^T
+// and dQ^T are N = 64 MMAs; dK and dV are N = 256.
+//
+// P^T and dS^T (bf16, 128 keys x 64 q rows, 16 KB) cross between the CTAs through
 // distributed shared memory: the producing compute warps store them straight into the
 // peer's buffer (st.shared::cluster, already in the 128B-swizzled K-major layout the
-// peer's MMA reads) and arrive on the peer's barrier.  The buffers are released back by
-// tcgen05.commit multicast to the other CTA plus the peer readers' remote arrivals.
-// CTA 0's ST is released as soon as its compute warps hold S^T in registers, so the next
-// slot's S^T runs while they compute the exponentials.
+// peer's MMA reads) and arrive on the peer's barrier.  A buffer goes back to its writer
+// once the peer's MMA has read it (tcgen05.commit multicast to the writer's CTA) and, on
+// CTA 1, once its compute warps have read P^T.
 //
-// dQ^T (fp32) leaves through TMEM -> shared memory (the slot's Q stage, free once dK has
-// consumed it) -> one TMA bulk reduce-add per warp into the head-major accumulator.
+// dQ^T (fp32) leaves through TMEM -> the staging buffer -> one TMA bulk reduce-add per
+// warp and half into the head-major accumulator.
 //
 // Units (key tiles) are claimed dynamically by CTA 0's producer and handed to both CTAs
 // through a unit ring whose slots every consumer of both CTAs releases.  Every wait is
@@ -41,39 +44,43 @@ using namespace bwd;
 struct PairCfg {
   static constexpr int HD = 256;
   static constexpr int BKV = 128;                   // keys per tile (TMEM lanes)
-  static constexpr int BQ = 128;                    // q rows per slot
+  static constexpr int BQ = 64;                     // q rows per slot
   static constexpr int KB = HD / 64;                // 64-wide d blocks
-  static constexpr int TILE_BYTES = BKV * HD * 2;   // K or V tile: 64 KB
-  static constexpr int SLOT_BYTES = BQ * HD * 2;    // Q or dO slot: 64 KB
-  static constexpr int X_BYTES = BKV * BQ * 2;      // P^T or dS^T: 32 KB, [2 q blocks][128 keys][128 B]
+  static constexpr int NST = 3;                     // Q / dO stages
+  static constexpr int TILE_BYTES = BKV * HD * 2;   // K or V tile: 64 KB, [4 d blocks][128 keys][128 B]
+  static constexpr int SLOT_BYTES = BQ * HD * 2;    // Q or dO slot: 32 KB, [4 d blocks][64 q][128 B]
+  static constexpr int X_BYTES = BKV * BQ * 2;      // P^T or dS^T: 16 KB, [128 keys][64 q]
+  static constexpr int STG_BYTES = 128 * BQ * 4;    // one dQ^T half: [4 warps][64 q][32 d] fp32
   static constexpr int SMEM_T = 0;                          // K (CTA 0) or V (CTA 1)
-  static constexpr int SMEM_S = SMEM_T + TILE_BYTES;        // 2 stages: Q (CTA 0) or dO (CTA 1)
-  static constexpr int SMEM_X = SMEM_S + 2 * SLOT_BYTES;    // received: dS^T (CTA 0) or P^T (CTA 1)
-  static constexpr int SMEM_STAT = SMEM_X + X_BYTES;        // 2 stages x 128 fp32: lse or Delta
-  static constexpr int SMEM_BYTES = SMEM_STAT + 2 * BQ * 4;
+  static constexpr int SMEM_S = SMEM_T + TILE_BYTES;        // Q (CTA 0) or dO (CTA 1) stages
+  static constexpr int SMEM_X = SMEM_S + NST * SLOT_BYTES;  // received: dS^T (CTA 0) / P^T (CTA 1), x2
+  static constexpr int SMEM_STG = SMEM_X + 2 * X_BYTES;     // dQ^T staging (CTA 0)
+  static constexpr int SMEM_STAT = SMEM_STG + STG_BYTES;    // NST x 64 fp32: lse or Delta
+  static constexpr int SMEM_BYTES = SMEM_STAT + NST * BQ * 4;
   static constexpr int WARP_DQ = 8;      // warps 8..11 (CTA 0)
   static constexpr int WARP_LOAD = 12;
   static constexpr int WARP_MMA = 13;    // CTA 0: S^T;  CTA 1: dP^T  (and TMEM owner)
   static constexpr int WARP_MMA2 = 14;   // CTA 0: dK, dQ^T;  CTA 1: dV
   static constexpr int NTHREADS = 15 * 32;
   static constexpr uint32_t TM_ACC = 0;      // dK (CTA 0) / dV (CTA 1): 256 columns
-  static constexpr uint32_t TM_ST = 256;     // S^T (CTA 0) / dP^T (CTA 1)
-  static constexpr uint32_t TM_XT = 384;     // dQ^T half (CTA 0)
+  static constexpr uint32_t TM_ST = 256;     // S^T / dP^T, two buffers of BQ columns
+  static constexpr uint32_t TM_XT = 384;     // dQ^T: d half h at TM_XT + h * BQ (CTA 0)
   static constexpr uint32_t TM_COLS = 512;
   static_assert(SMEM_BYTES <= 227 * 1024 - 1024, "shared memory budget");
+  static_assert(TM_XT + 2 * BQ <= TM_COLS, "TMEM budget");
 };
 
 // The same barrier struct sits at the same offset in both CTAs, so a barrier of the peer
 // is addressed by mapping the local one (mapa) or by a multicast commit.
 struct PairBars {
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];  // unit_empty used in CTA 0 only
-  uint64_t t_full, t_empty;           // K / V tile
-  uint64_t s_full[2], s_empty[2];     // Q / dO (+ lse / Delta) stages
-  uint64_t mm_full, mm_free;          // S^T (CTA 0) / dP^T (CTA 1) in TMEM, and its release
-  uint64_t x_full;                    // the peer's P^T (CTA 1) / dS^T (CTA 0) has arrived
-  uint64_t x_free;                    // CTA 0: CTA 1 is done with P^T;  CTA 1: CTA 0 with dS^T
-  uint64_t dq_full, dq_empty;         // dQ^T half in XT (CTA 0)
-  uint64_t acc_full, acc_empty;       // dK / dV accumulators
+  uint64_t t_full, t_empty;                       // K / V tile
+  uint64_t s_full[PairCfg::NST], s_empty[PairCfg::NST];   // Q / dO (+ lse / Delta) stages
+  uint64_t mm_full[2], mm_free[2];   // S^T (CTA 0) / dP^T (CTA 1) buffers in TMEM
+  uint64_t x_full[2];                // the peer's P^T (CTA 1) / dS^T (CTA 0) has arrived
+  uint64_t x_free[2];                // CTA 0: CTA 1 is done with P^T;  CTA 1: CTA 0 with dS^T
+  uint64_t dq_full, dq_empty;        // dQ^T in XT (CTA 0)
+  uint64_t acc_full, acc_empty;      // dK / dV accumulators
   uint64_t drain, never;
 };
 
@@ -101,7 +108,7 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
                         const __grid_constant__ CUtensorMap map_do,
                         const __grid_constant__ CUtensorMap map_dq, const BwdParams prm) {
   using Cfg = PairCfg;
-  constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV;
+  constexpr int KB = Cfg::KB, BQ = Cfg::BQ, BKV = Cfg::BKV, NST = Cfg::NST;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ PairBars bars;
   __shared__ uint32_t tmem_base_s;
@@ -123,16 +130,18 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
     }
     mbar_init(&bars.t_full, 1);
     mbar_init(&bars.t_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&bars.s_full[s], 1);
-      // CTA 0: 8 compute warps (lse read) + 4 dQ warps (dQ^T staged out of the stage);
-      // CTA 1: 8 compute warps (Delta read, dP^T complete) + the dV commit
-      mbar_init(&bars.s_empty[s], rank == 0 ? 8 + 4 : 8 + 1);
+      // 8 compute warps (lse / Delta read) + the commit after the last MMA reading the
+      // stage (dK on CTA 0, dV on CTA 1)
+      mbar_init(&bars.s_empty[s], 8 + 1);
     }
-    mbar_init(&bars.mm_full, 1);
-    mbar_init(&bars.mm_free, 8);
-    mbar_init(&bars.x_full, 8);                       // the peer's 8 compute warps
-    mbar_init(&bars.x_free, rank == 0 ? 1 + 8 : 1);   // CTA 1's dV commit + its compute warps
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.mm_full[b], 1);
+      mbar_init(&bars.mm_free[b], 8);
+      mbar_init(&bars.x_full[b], 8);                       // the peer's 8 compute warps
+      mbar_init(&bars.x_free[b], rank == 0 ? 1 + 8 : 1);   // CTA 1: dV commit + compute warps
+    }
     mbar_init(&bars.dq_full, 1);
     mbar_init(&bars.dq_empty, 4);
     mbar_init(&bars.acc_full, 1);
@@ -165,7 +174,8 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t s_it = 0, t_fills = 0;
-      uint32_t s_fills[2] = {0, 0};
+      uint32_t s_fills[NST];
+      for (int s = 0; s < NST; ++s) s_fills[s] = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int slot = k % kUnitRing;
@@ -188,13 +198,13 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         }
         if (idx < 0) break;
         const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
-        // the unit's K (CTA 0) or V (CTA 1) tile, in 64-key boxes
+        // the unit's K (CTA 0) or V (CTA 1) tile
         if (t_fills > 0) ok = mbar_wait(&bars.t_empty, (t_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.t_full, Cfg::TILE_BYTES);
         for (int hb = 0; hb < BKV / prm.kv_box; ++hb) {
-          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * prm.kv_box, u.b, prm.S, prm.B, prm.D,
-                                             prm.kv_shard_major);
+          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * prm.kv_box, u.b, prm.S,
+                                             prm.B, prm.D, prm.kv_shard_major);
           for (int kb = 0; kb < KB; ++kb)
             tma_load_3d(smem + Cfg::SMEM_T + kb * BKV * 128 + hb * prm.kv_box * 128,
                         rank == 0 ? &map_k : &map_v, &bars.t_full, kb * 64, u.g, krow);
@@ -203,8 +213,8 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         // the q slots: Q + lse (CTA 0) or dO + Delta (CTA 1)
         SlotWalk w;
         for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
-          const int st = int(s_it & 1);
-          const uint32_t use = s_it >> 1;
+          const int st = int(s_it % NST);
+          const uint32_t use = s_it / NST;
           if (use > 0) ok = mbar_wait(&bars.s_empty[st], (use - 1) & 1, wctx);
           if (!ok) break;
           const int32_t h = u.g * prm.G + w.e;
@@ -224,26 +234,28 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
       if (!ok) {
         const uint64_t lim = 1000000000ull;
         if (t_fills > 0) mbar_drain(&bars.t_full, (t_fills - 1) & 1, lim);
-        for (int s = 0; s < 2; ++s)
+        for (int s = 0; s < NST; ++s)
           if (s_fills[s] > 0) mbar_drain(&bars.s_full[s], (s_fills[s] - 1) & 1, lim);
       }
     }
   } else if (warp == Cfg::WARP_MMA || warp == Cfg::WARP_MMA2) {
     // ------------------------------------------------------------ MMA issuers
-    //  thread A (WARP_MMA): S^T = K Q^T (CTA 0) or dP^T = V dO^T (CTA 1) into ST, each as
-    //    soon as the slot's stage is loaded and the compute warps have read the previous
-    //    product out of ST;
-    //  thread B (WARP_MMA2): CTA 0: dK += dS^T Q, then dQ^T = K^T dS^T in two 128-row d
-    //    halves through XT;  CTA 1: dV += P^T dO.  Both read the operand the peer stored
-    //    into this CTA's X buffer, and release it to the peer by a multicast commit.
+    //  thread A (WARP_MMA): S^T = K Q^T (CTA 0) or dP^T = V dO^T (CTA 1) into ST buffer
+    //    j % 2, as soon as the slot's stage is loaded and the compute warps have read
+    //    slot j-2's product out of that buffer;
+    //  thread B (WARP_MMA2): CTA 0: dK += dS^T Q, then both 128-row halves of
+    //    dQ^T = K^T dS^T into XT;  CTA 1: dV += P^T dO.  Both read the operand the peer
+    //    stored into this CTA's exchange buffer j % 2, and hand it back to the peer with a
+    //    multicast commit.
     if (lane == 0) {
       const bool role_a = warp == Cfg::WARP_MMA;
       const uint32_t idesc_s = idesc_bf16(128, BQ, false, false);      // S^T, dP^T
       const uint32_t idesc_acc = idesc_bf16(128, 256, false, true);    // dK, dV (N = d = 256)
       const uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);       // dQ^T half
-      uint32_t t_ph = 0, q_it = 0, x_ph = 0;
-      uint32_t s_uses[2] = {0, 0};
-      uint32_t mmfree_waits = 0, dq_commits = 0, dq_waits = 0, acc_commits = 0;
+      uint32_t t_ph = 0, q_it = 0;
+      uint32_t s_uses[NST];
+      for (int s = 0; s < NST; ++s) s_uses[s] = 0;
+      uint32_t dq_commits = 0, acc_commits = 0;
       bool ok = true;
       if (prm.inject_stall) ok = mbar_wait(&bars.never, 0, wctx);
       for (int k = 0; ok; ++k) {
@@ -261,57 +273,55 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         SlotWalk w;
         for (bool more = walk_first(prm, u.n, w), j0 = true; more && ok;
              more = walk_next(prm, u.n, w), j0 = false) {
-          const int st = int(q_it & 1);
+          const int st = int(q_it % NST);
+          const int xb = int(q_it & 1);                 // ST / exchange buffer of this slot
           const uint32_t sSt = sS + uint32_t(st * Cfg::SLOT_BYTES);
+          const uint32_t sXb = sX + uint32_t(xb * Cfg::X_BYTES);
           if (role_a) {
             ok = mbar_wait(&bars.s_full[st], s_uses[st] & 1, wctx);
             ++s_uses[st];
-            if (ok && q_it > 0) ok = mbar_wait(&bars.mm_free, mmfree_waits++ & 1, wctx);
+            if (ok && q_it >= 2) ok = mbar_wait(&bars.mm_free[xb], ((q_it >> 1) - 1) & 1, wctx);
             if (!ok) break;
             tc_fence_after();
             for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma_ss(tmem + Cfg::TM_ST, sdesc_sw128(sT + kb * BKV * 128 + ks * 32, 16, 1024),
+                mma_ss(tmem + Cfg::TM_ST + uint32_t(xb * BQ),
+                       sdesc_sw128(sT + kb * BKV * 128 + ks * 32, 16, 1024),
                        sdesc_sw128(sSt + kb * BQ * 128 + ks * 32, 16, 1024), idesc_s, (kb | ks) != 0);
-            mma_commit(&bars.mm_full);
+            mma_commit(&bars.mm_full[xb]);
           } else {
             // the peer's operand for this slot: dS^T (CTA 0) or P^T (CTA 1)
-            ok = mbar_wait_cluster(&bars.x_full, x_ph, wctx);
-            x_ph ^= 1;
+            ok = mbar_wait_cluster(&bars.x_full[xb], (q_it >> 1) & 1, wctx);
             if (ok && j0 && acc_commits > 0)
               ok = mbar_wait(&bars.acc_empty, (acc_commits - 1) & 1, wctx);
             if (!ok) break;
             tc_fence_after();
-            // dK += dS^T Q  /  dV += P^T dO: A = X (K-major, 64-q blocks), B = the stage
-            // (MN-major, N = 256 over four 64-wide d blocks)
+            // dK += dS^T Q  /  dV += P^T dO: A = the exchange buffer (K-major, one 64-q
+            // block), B = the stage (MN-major, N = 256 over four 64-wide d blocks)
 #pragma unroll
             for (int ks = 0; ks < BQ / 16; ++ks)
-              mma_ss(tmem + Cfg::TM_ACC, sdesc_sw128(sX + (ks >> 2) * (BKV * 128) + (ks & 3) * 32, 16, 1024),
+              mma_ss(tmem + Cfg::TM_ACC, sdesc_sw128(sXb + ks * 32, 16, 1024),
                      sdesc_sw128(sSt + ks * 2048, BQ * 128, 1024), idesc_acc, !j0 || (ks > 0));
+            mma_commit(&bars.s_empty[st]);              // the stage's last MMA reader
             if (rank == 0) {
-              for (int hh = 0; hh < 2 && ok; ++hh) {
-                if (dq_commits > dq_waits) {
-                  ok = mbar_wait(&bars.dq_empty, dq_waits & 1, wctx);
-                  ++dq_waits;
-                  if (!ok) break;
-                  tc_fence_after();
-                }
-                // dQ^T rows 128hh .. 128hh+127: A = K^T (MN-major, d blocks 2hh, 2hh+1),
-                // B = dS^T (MN-major, 64-q blocks), K = the 128 keys
+              // dQ^T rows 128hh .. 128hh+127: A = K^T (MN-major, d blocks 2hh, 2hh+1),
+              // B = dS^T (MN-major: the 64 q of each key row), K = the 128 keys
+              if (dq_commits > 0) {
+                ok = mbar_wait(&bars.dq_empty, (dq_commits - 1) & 1, wctx);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
                 for (int ks = 0; ks < BKV / 16; ++ks)
-                  mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sT + (2 * hh) * (BKV * 128) + ks * 2048, BKV * 128, 1024),
-                         sdesc_sw128(sX + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
-                mma_commit(&bars.dq_full);
-                ++dq_commits;
-              }
-              if (!ok) break;
-              mma_commit_multicast(&bars.x_free, uint16_t(1u << peer));   // dS^T buffer free
-            } else {
-              mma_commit_multicast(&bars.x_free, uint16_t(1u << peer));   // P^T buffer free
-              mma_commit(&bars.s_empty[st]);                               // dO of the stage
+                  mma_ss(tmem + Cfg::TM_XT + uint32_t(hh * BQ),
+                         sdesc_sw128(sT + (2 * hh) * (BKV * 128) + ks * 2048, BKV * 128, 1024),
+                         sdesc_sw128(sXb + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
+              mma_commit(&bars.dq_full);
+              ++dq_commits;
             }
+            mma_commit_multicast(&bars.x_free[xb], uint16_t(1u << peer));   // buffer back
           }
           ++q_it;
         }
@@ -330,15 +340,15 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
     __syncwarp();
   } else if (warp >= Cfg::WARP_DQ) {
     // ------------------------------------------------------------ dQ warps (CTA 0)
-    // Each dQ^T half (TMEM lane = d within the half, column = q row) is staged as four
-    // [128 q][32 d] fp32 boxes (one per warp, 128-byte rows, 128-byte swizzle) in the
-    // slot's Q stage -- every MMA reading Q has completed once dQ^T exists -- and reduced
-    // into the accumulator by one TMA bulk reduce-add per warp.  The second half reuses
-    // the box after the first half's reduce has read it.
+    // Each dQ^T half of a slot (TMEM lane = d within the half, column = q row) is staged
+    // as four [64 q][32 d] fp32 boxes (one per warp, 128-byte rows, 128-byte swizzle) in
+    // the staging buffer and reduced into the accumulator by one TMA bulk reduce-add per
+    // warp; the second half reuses the box after the first half's reduce has read it.
     if (rank == 0) {
       const int qw = warp - Cfg::WARP_DQ;
       const uint32_t tXT = tmem + Cfg::TM_XT + (uint32_t(qw * 32) << 16);
-      uint32_t dq_ph = 0, q_it = 0;
+      uint8_t* box = smem + Cfg::SMEM_STG + qw * (BQ * 128);
+      uint32_t dq_ph = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int slot = k % kUnitRing;
@@ -351,32 +361,30 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
         SlotWalk w;
         for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
-          const int st = int(q_it & 1);
-          uint8_t* box = smem + Cfg::SMEM_S + st * Cfg::SLOT_BYTES + qw * (BQ * 128);
+          ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
+          dq_ph ^= 1;
+          if (!ok) break;
+          tc_fence_after();
           const int32_t h = u.g * prm.G + w.e;
           const int32_t row0 =
               int32_t((int64_t(w.r - prm.shard_begin) * prm.B + u.b) * twoC + int64_t(w.i) * BQ);
           for (int hh = 0; hh < 2; ++hh) {
-            ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
-            dq_ph ^= 1;
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int t = 0; t < BQ / 32; ++t) {
-              uint32_t v[32];
-              tmem_ld32(tXT + t * 32, v);
-              tmem_ld_wait();
-              if (t + 1 == BQ / 32) {          // the half is in registers: XT may be reused
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.dq_empty);
-              }
-              const uint32_t within = uint32_t(lane & 3) * 4;
+            uint32_t v[2][32];
+            tmem_ld32(tXT + uint32_t(hh * BQ), v[0]);
+            tmem_ld32(tXT + uint32_t(hh * BQ + 32), v[1]);
+            tmem_ld_wait();
+            if (hh == 1) {                     // all of dQ^T read: XT may take the next
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars.dq_empty);
+            }
+            const uint32_t within = uint32_t(lane & 3) * 4;
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
 #pragma unroll
               for (int c = 0; c < 32; ++c)
                 *reinterpret_cast<uint32_t*>(box + sw128_offset(uint32_t(t * 32 + c), uint32_t(lane >> 2)) +
-                                             within) = v[c];
-            }
+                                             within) = v[t][c];
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -386,9 +394,6 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
             }
             __syncwarp();
           }
-          if (!ok) break;
-          if (lane == 0) mbar_arrive(&bars.s_empty[st]);
-          ++q_it;
         }
       }
       if (lane == 0) bulk_wait_group0();
@@ -396,25 +401,22 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ compute warps
-    // group hg = warp / 4 handles q rows 64hg .. 64hg+63 of each slot (contiguous
-    // positions: a 64-row half never straddles a zigzag chunk); thread = key row.
+    // group hg = warp / 4 handles q rows 32hg .. 32hg+31 of each 64-row slot (contiguous
+    // positions: a 64-row slot lies inside one zigzag chunk); thread = key row.
     //  CTA 0: P^T = exp(scale S^T - lse) (masked) -> the peer's P^T buffer.
     //  CTA 1: dS^T = P^T (dP^T - Delta) -> the peer's dS^T buffer.
     const int hg = warp / 4;
     const int qw = warp % 4;
     const int row = qw * 32 + lane;
     const uint32_t lane_addr = uint32_t(qw * 32) << 16;
-    const uint32_t tM = tmem + Cfg::TM_ST + 64 * hg + lane_addr;
-    const uint32_t x_peer = peer_addr(smem + Cfg::SMEM_X + hg * (BKV * 128), peer);
-    const uint8_t* x_local = smem + Cfg::SMEM_X + hg * (BKV * 128);
     const float* stat = reinterpret_cast<const float*>(smem + Cfg::SMEM_STAT);
-    uint32_t q_it = 0, mm_ph = 0, x_ph = 0, xf_waits = 0, acc_ph = 0;
-    uint32_t s_uses[2] = {0, 0};
+    uint32_t q_it = 0, acc_ph = 0;
+    uint32_t s_uses[NST];
+    for (int s = 0; s < NST; ++s) s_uses[s] = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int slot = k % kUnitRing;
-      ok = mbar_wait_cluster(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bars.unit_full[slot], (k / kUnitRing) & 1, wctx));
       if (!ok) break;
       const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
       __syncwarp();
@@ -429,78 +431,73 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
       SlotWalk w;
       for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
         ++nslots;
-        const int st = int(q_it & 1);
+        const int st = int(q_it % NST);
+        const int xb = int(q_it & 1);
+        const uint32_t ph = (q_it >> 1) & 1;              // phase of the slot's buffers
         ok = warp_wait_b(&bars.s_full[st], s_uses[st] & 1, wctx);
         ++s_uses[st];
         if (!ok) break;
-        const float* stat_c = stat + st * BQ + 64 * hg;
-        // ---- this slot's ST product (S^T or dP^T), 64 columns per thread
-        ok = warp_wait_b(&bars.mm_full, mm_ph, wctx);
-        mm_ph ^= 1;
+        const float* stat_c = stat + st * BQ + 32 * hg;
+        // ---- this slot's product (S^T or dP^T), 32 columns per thread
+        ok = warp_wait_b(&bars.mm_full[xb], ph, wctx);
         if (!ok) break;
         tc_fence_after();
-        uint32_t sv[2][32];
-        tmem_ld32(tM, sv[0]);
-        tmem_ld32(tM + 32, sv[1]);
+        uint32_t sv[32];
+        tmem_ld32(tmem + Cfg::TM_ST + uint32_t(xb * BQ + 32 * hg) + lane_addr, sv);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.mm_free);       // ST may take the next product
-        uint32_t pk[2][16];
+        if (lane == 0) mbar_arrive(&bars.mm_free[xb]);    // the buffer may take slot j+2
+        uint32_t pk[16];
         if (rank == 0) {
           // P^T: columns c < nvis_lo lie above the diagonal for this key
-          const int64_t p0 = zz_pos(prm.C, prm.D, w.r, int64_t(w.i) * BQ + 64 * hg);
+          const int64_t p0 = zz_pos(prm.C, prm.D, w.r, int64_t(w.i) * BQ + 32 * hg);
           const int nvis_lo = prm.causal ? int(key - p0) : 0;
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c0 = cc * 32 + 2 * e;
-              const float x0 = fmaf(__uint_as_float(sv[cc][2 * e]), prm.scale_log2, -stat_c[c0] * kLog2e);
-              const float x1 = fmaf(__uint_as_float(sv[cc][2 * e + 1]), prm.scale_log2, -stat_c[c0 + 1] * kLog2e);
-              pk[cc][e] = pack_bf16x2(c0 < nvis_lo ? 0.f : ex2_approx(x0),
-                                      c0 + 1 < nvis_lo ? 0.f : ex2_approx(x1));
-            }
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 2 * e;
+            const float x0 = fmaf(__uint_as_float(sv[c0]), prm.scale_log2, -stat_c[c0] * kLog2e);
+            const float x1 = fmaf(__uint_as_float(sv[c0 + 1]), prm.scale_log2, -stat_c[c0 + 1] * kLog2e);
+            pk[e] = pack_bf16x2(c0 < nvis_lo ? 0.f : ex2_approx(x0),
+                                c0 + 1 < nvis_lo ? 0.f : ex2_approx(x1));
+          }
         } else {
-          // dS^T needs P^T of this slot from the peer
-          ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bars.x_full, x_ph, wctx));
-          x_ph ^= 1;
+          // dS^T needs this slot's P^T from the peer
+          ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bars.x_full[xb], ph, wctx));
           if (!ok) break;
-          uint4 pv[8];
+          const uint8_t* x_local = smem + Cfg::SMEM_X + xb * Cfg::X_BYTES;
+          uint4 pv[4];
 #pragma unroll
-          for (int m = 0; m < 8; ++m)
-            pv[m] = *reinterpret_cast<const uint4*>(x_local + sw128_offset(uint32_t(row), uint32_t(m)));
+          for (int m = 0; m < 4; ++m)
+            pv[m] = *reinterpret_cast<const uint4*>(x_local + sw128_offset(uint32_t(row), uint32_t(4 * hg + m)));
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(peer_addr(&bars.x_free, peer));   // P^T read
+          if (lane == 0) mbar_arrive_cluster(peer_addr(&bars.x_free[xb], peer));   // P^T read
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
+          for (int m = 0; m < 4; ++m) {
             const uint32_t pw[4] = {pv[m].x, pv[m].y, pv[m].z, pv[m].w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-              const int c0 = 8 * m + 2 * t;            // column within the group's 64
-              const float p0f = __uint_as_float(pw[t] << 16);
-              const float p1f = __uint_as_float(pw[t] & 0xFFFF0000u);
-              pk[c0 >> 5][(c0 & 31) >> 1] =
-                  pack_bf16x2(p0f * (__uint_as_float(sv[c0 >> 5][c0 & 31]) - stat_c[c0]),
-                              p1f * (__uint_as_float(sv[c0 >> 5][(c0 & 31) + 1]) - stat_c[c0 + 1]));
+              const int c0 = 8 * m + 2 * t;
+              pk[4 * m + t] =
+                  pack_bf16x2(__uint_as_float(pw[t] << 16) * (__uint_as_float(sv[c0]) - stat_c[c0]),
+                              __uint_as_float(pw[t] & 0xFFFF0000u) * (__uint_as_float(sv[c0 + 1]) - stat_c[c0 + 1]));
             }
           }
         }
-        // the peer's buffer must be free of the previous slot's operand
-        if (q_it > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bars.x_free, xf_waits & 1, wctx));
-          ++xf_waits;
+        // the peer's buffer must be done with slot j-2's operand
+        if (q_it >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bars.x_free[xb], ph ^ 1u, wctx));
           if (!ok) break;
         }
+        const uint32_t x_peer = peer_addr(smem + Cfg::SMEM_X + xb * Cfg::X_BYTES, peer);
 #pragma unroll
-        for (int m = 0; m < 8; ++m)
-          st_cluster_v4(x_peer + sw128_offset(uint32_t(row), uint32_t(m)),
-                        make_uint4(pk[m >> 2][4 * (m & 3)], pk[m >> 2][4 * (m & 3) + 1],
-                                   pk[m >> 2][4 * (m & 3) + 2], pk[m >> 2][4 * (m & 3) + 3]));
+        for (int m = 0; m < 4; ++m)
+          st_cluster_v4(x_peer + sw128_offset(uint32_t(row), uint32_t(4 * hg + m)),
+                        make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]));
         fence_proxy_async_cluster();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_cluster(peer_addr(&bars.x_full, peer));
+          mbar_arrive_cluster(peer_addr(&bars.x_full[xb], peer));
           mbar_arrive(&bars.s_empty[st]);             // lse / Delta of the stage consumed
         }
         ++q_it;

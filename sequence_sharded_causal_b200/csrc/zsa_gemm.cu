@@ -9,6 +9,9 @@
 // belong: Q, K and V columns of the shard's heads (bf16, overwritten), or an fp32
 // accumulator that sums the output projection's per-step partials.
 //
+// Any T; N a multiple of 32; K a multiple of 8: tiles past the edges load zeros (TMA
+// out-of-bounds fill) and the epilogue stores only rows < T and 32-column chunks < N.
+//
 // Kernel: persistent CTAs over 128 x 128 output tiles (tile t -> m block t % MT, n block
 // t / MT: CTAs running together share one column block of W_s in L2).  One TMA warp
 // streams [128 m][64 k] tiles of X (K-major) and [64 k][128 n] tiles of W_s (two 64-wide
@@ -91,7 +94,7 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
   const uint32_t tmem = tmem_base_s;
   const WaitCtx wctx{&abort_s, prm.status, prm.wait_limit_ns};
   const int32_t n_tiles = prm.mt * prm.nt;
-  const int32_t kblocks = int32_t(prm.K / Cfg::BK);
+  const int32_t kblocks = int32_t((prm.K + Cfg::BK - 1) / Cfg::BK);
 
   if (warp == Cfg::WARP_LOAD) {
     if (lane == 0) {
@@ -162,12 +165,14 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
       tc_fence_after();
       const int64_t m = int64_t(t % prm.mt) * Cfg::BM + row;
       const int64_t n0 = int64_t(t / prm.mt) * Cfg::BN;
+      const bool row_in = m < prm.T;
 #pragma unroll 1
       for (int c = 0; c < Cfg::BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + uint32_t(acc * Cfg::BN + c * 32) + lane_addr, v);
         tmem_ld_wait();
         int64_t col = n0 + c * 32;
+        if (!row_in || col >= prm.N) continue;       // past the output's edge
         int si = 0;
         while (si + 1 < prm.n_segs && col >= prm.segs[si].col_end) ++si;
         const ProjSegment& sg = prm.segs[si];
@@ -223,8 +228,8 @@ int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
   }
   GemmParams p;
   p.T = a.T; p.N = a.N; p.K = a.K;
-  p.mt = int32_t(a.T / Cfg::BM);
-  p.nt = int32_t(a.N / Cfg::BN);
+  p.mt = int32_t((a.T + Cfg::BM - 1) / Cfg::BM);
+  p.nt = int32_t((a.N + Cfg::BN - 1) / Cfg::BN);
   p.n_segs = a.n_segs;
   for (int i = 0; i < a.n_segs; ++i) p.segs[i] = a.segs[i];
   p.status = a.status;

@@ -109,8 +109,8 @@ def test_tsp_project_argument_errors():
 
     def rc(T=256, K=128, N=256, x=16, ldx=128, w=16, ldw=256, segs=sp, n=1, ws=256):
         return L.zsa_tsp_project(T, K, N, x, ldx, w, ldw, segs, n, ws, None)
-    assert rc(T=100) == zsa.ZSA_ERR_SHAPE          # T % 128
-    assert rc(K=96) == zsa.ZSA_ERR_SHAPE           # K % 64
+    assert rc(N=250) == zsa.ZSA_ERR_SHAPE          # N % 32
+    assert rc(K=100) == zsa.ZSA_ERR_SHAPE          # K % 8
     assert rc(x=None) == zsa.ZSA_ERR_INVALID
     assert rc(x=24) == zsa.ZSA_ERR_INVALID         # misaligned
     assert rc(ldx=100) == zsa.ZSA_ERR_INVALID      # ldx < K

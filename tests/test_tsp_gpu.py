@@ -36,7 +36,8 @@ def _rand(shape, seed, scale=1.0):
 
 
 @pytest.mark.parametrize("T,K,N", [(128, 64, 128), (256, 512, 384), (1024, 4096, 768),
-                                   (384, 1280, 1024)])
+                                   (384, 1280, 1024),
+                                   (200, 72, 160)])    # ragged: T, N, K past the tile edges
 def test_project_bf16_matches_oracle(oracle, T, K, N):
     x, w = _rand((T, K), 1), _rand((K, N), 2, 0.05)
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
