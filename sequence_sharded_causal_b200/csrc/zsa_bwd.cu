@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         if (!ok) break;
         mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
         for (int hb = 0; hb < BKV / prm.kv_box; ++hb) {
-          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * prm.kv_box, u.b, prm.S, prm.B, prm.D,
+          const int32_t krow = kv_tensor_row(u.n * BKV + hb * prm.kv_box, u.b, int32_t(prm.S), int32_t(prm.C), prm.B, prm.D,
                                              prm.kv_shard_major);
           for (int kb = 0; kb < KB; ++kb) {
             tma_load_3d(smem + Cfg::SMEM_K + kb * BKV * 128 + hb * prm.kv_box * 128, &map_k, &bars.kv_full,
@@ -592,7 +592,8 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
       tc_fence_after();
       const uint32_t tAcc = tmem + (hgrp == 0 ? Cfg::TM_DV : Cfg::TM_DK) + lane_addr;
       const float mul = hgrp == 0 ? 1.0f : prm.scale;
-      const int64_t krow = kv_tensor_row(key, u.b, prm.S, prm.B, prm.D, prm.kv_shard_major);
+      const int64_t krow = kv_tensor_row(int32_t(key), u.b, int32_t(prm.S), int32_t(prm.C), prm.B, prm.D,
+                                           prm.kv_shard_major);
       __nv_bfloat16* dst = (hgrp == 0 ? prm.dv : prm.dk) + (krow * prm.Hkv + u.g) * HD;
       // a key tile no query of the launch's shards sees has no MMA behind its
       // accumulators: its dK / dV rows are zero

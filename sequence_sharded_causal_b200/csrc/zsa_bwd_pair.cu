@@ -79,7 +79,7 @@ struct PairBars {
   uint64_t mm_full[2], mm_free[2];   // S^T (CTA 0) / dP^T (CTA 1) buffers in TMEM
   uint64_t x_full[2];                // the peer's P^T (CTA 1) / dS^T (CTA 0) has arrived
   uint64_t x_free[2];                // CTA 0: CTA 1 is done with P^T;  CTA 1: CTA 0 with dS^T
-  uint64_t dq_full, dq_empty;        // dQ^T in XT (CTA 0)
+  uint64_t dq_full[2], dq_empty[2];  // dQ^T half h in XT (CTA 0), per half
   uint64_t acc_full, acc_empty;      // dK / dV accumulators
   uint64_t drain, never;
 };
@@ -142,8 +142,10 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
       mbar_init(&bars.x_full[b], 8);                       // the peer's 8 compute warps
       mbar_init(&bars.x_free[b], rank == 0 ? 1 + 8 : 1);   // CTA 1: dV commit + compute warps
     }
-    mbar_init(&bars.dq_full, 1);
-    mbar_init(&bars.dq_empty, 4);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars.dq_full[h], 1);
+      mbar_init(&bars.dq_empty[h], 4);
+    }
     mbar_init(&bars.acc_full, 1);
     mbar_init(&bars.acc_empty, 8);
     mbar_init(&bars.drain, 2);
@@ -203,8 +205,8 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         if (!ok) break;
         mbar_expect_tx(&bars.t_full, Cfg::TILE_BYTES);
         for (int hb = 0; hb < BKV / prm.kv_box; ++hb) {
-          const int32_t krow = kv_tensor_row(int64_t(u.n) * BKV + hb * prm.kv_box, u.b, prm.S,
-                                             prm.B, prm.D, prm.kv_shard_major);
+          const int32_t krow = kv_tensor_row(u.n * BKV + hb * prm.kv_box, u.b, int32_t(prm.S),
+                                             int32_t(prm.C), prm.B, prm.D, prm.kv_shard_major);
           for (int kb = 0; kb < KB; ++kb)
             tma_load_3d(smem + Cfg::SMEM_T + kb * BKV * 128 + hb * prm.kv_box * 128,
                         rank == 0 ? &map_k : &map_v, &bars.t_full, kb * 64, u.g, krow);
@@ -306,19 +308,23 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
             mma_commit(&bars.s_empty[st]);              // the stage's last MMA reader
             if (rank == 0) {
               // dQ^T rows 128hh .. 128hh+127: A = K^T (MN-major, d blocks 2hh, 2hh+1),
-              // B = dS^T (MN-major: the 64 q of each key row), K = the 128 keys
-              if (dq_commits > 0) {
-                ok = mbar_wait(&bars.dq_empty, (dq_commits - 1) & 1, wctx);
-                if (!ok) break;
-                tc_fence_after();
-              }
-              for (int hh = 0; hh < 2; ++hh)
+              // B = dS^T (MN-major: the 64 q of each key row), K = the 128 keys.  Each
+              // half has its own TMEM columns and hand-off, so half 0 of this slot only
+              // waits for half 0 of the previous one to be read out.
+              for (int hh = 0; hh < 2 && ok; ++hh) {
+                if (dq_commits > 0) {
+                  ok = mbar_wait(&bars.dq_empty[hh], (dq_commits - 1) & 1, wctx);
+                  if (!ok) break;
+                  tc_fence_after();
+                }
 #pragma unroll
                 for (int ks = 0; ks < BKV / 16; ++ks)
                   mma_ss(tmem + Cfg::TM_XT + uint32_t(hh * BQ),
                          sdesc_sw128(sT + (2 * hh) * (BKV * 128) + ks * 2048, BKV * 128, 1024),
                          sdesc_sw128(sXb + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
-              mma_commit(&bars.dq_full);
+                mma_commit(&bars.dq_full[hh]);
+              }
+              if (!ok) break;
               ++dq_commits;
             }
             mma_commit_multicast(&bars.x_free[xb], uint16_t(1u << peer));   // buffer back
@@ -361,23 +367,20 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
         SlotWalk w;
         for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
-          ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
-          dq_ph ^= 1;
-          if (!ok) break;
-          tc_fence_after();
           const int32_t h = u.g * prm.G + w.e;
           const int32_t row0 =
               int32_t((int64_t(w.r - prm.shard_begin) * prm.B + u.b) * twoC + int64_t(w.i) * BQ);
           for (int hh = 0; hh < 2; ++hh) {
+            ok = warp_wait_b(&bars.dq_full[hh], dq_ph, wctx);
+            if (!ok) break;
+            tc_fence_after();
             uint32_t v[2][32];
             tmem_ld32(tXT + uint32_t(hh * BQ), v[0]);
             tmem_ld32(tXT + uint32_t(hh * BQ + 32), v[1]);
             tmem_ld_wait();
-            if (hh == 1) {                     // all of dQ^T read: XT may take the next
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&bars.dq_empty);
-            }
+            tc_fence_before();                 // the half is in registers: its columns
+            __syncwarp();                      // may take the next slot's half
+            if (lane == 0) mbar_arrive(&bars.dq_empty[hh]);
             const uint32_t within = uint32_t(lane & 3) * 4;
 #pragma unroll
             for (int t = 0; t < 2; ++t)
@@ -394,6 +397,7 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
             }
             __syncwarp();
           }
+          dq_ph ^= 1;
         }
       }
       if (lane == 0) bulk_wait_group0();
@@ -510,7 +514,8 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const float mul = rank == 0 ? prm.scale : 1.0f;
-      const int64_t krow = kv_tensor_row(key, u.b, prm.S, prm.B, prm.D, prm.kv_shard_major);
+      const int64_t krow = kv_tensor_row(int32_t(key), u.b, int32_t(prm.S), int32_t(prm.C), prm.B, prm.D,
+                                           prm.kv_shard_major);
       __nv_bfloat16* dst = (rank == 0 ? prm.dk : prm.dv) + (krow * prm.Hkv + u.g) * Cfg::HD + 128 * hg;
       const bool empty = nslots == 0;   // no query of the launch's shards sees this tile
 #pragma unroll 1

@@ -225,12 +225,20 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.k_full[st], Cfg::KV_BYTES);
-            for (int hb = 0; hb < BK / prm.kv_box; ++hb) {
-              const int32_t krow = kv_tensor_row(int64_t(n) * BK + hb * prm.kv_box, u.b, prm.S, prm.B,
-                                                 prm.D, prm.kv_shard_major);
+            if (prm.kv_box == BK) {       // the tile's rows are contiguous: one box per d block
+              const int32_t krow = kv_tensor_row(n * BK, u.b, int32_t(prm.S), int32_t(prm.C),
+                                                 prm.B, prm.D, prm.kv_shard_major);
               for (int kb = 0; kb < KB; ++kb)
-                tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128 + hb * prm.kv_box * 128,
-                            &map_k, &bars.k_full[st], kb * 64, u.g, krow);
+                tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128, &map_k,
+                            &bars.k_full[st], kb * 64, u.g, krow);
+            } else {                      // 64-key boxes, one zigzag chunk each
+              for (int hb = 0; hb < BK / 64; ++hb) {
+                const int32_t krow = kv_tensor_row(n * BK + hb * 64, u.b, int32_t(prm.S),
+                                                   int32_t(prm.C), prm.B, prm.D, prm.kv_shard_major);
+                for (int kb = 0; kb < KB; ++kb)
+                  tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
+                              &map_k, &bars.k_full[st], kb * 64, u.g, krow);
+              }
             }
             ++k_fills[st];
           }
@@ -241,12 +249,20 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.v_full[st], Cfg::KV_BYTES);
-            for (int hb = 0; hb < BK / prm.kv_box; ++hb) {
-              const int32_t vrow = kv_tensor_row(int64_t(n - 1) * BK + hb * prm.kv_box, u.b, prm.S, prm.B,
-                                                 prm.D, prm.kv_shard_major);
+            if (prm.kv_box == BK) {
+              const int32_t vrow = kv_tensor_row((n - 1) * BK, u.b, int32_t(prm.S), int32_t(prm.C),
+                                                 prm.B, prm.D, prm.kv_shard_major);
               for (int kb = 0; kb < KB; ++kb)
-                tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128 + hb * prm.kv_box * 128,
-                            &map_v, &bars.v_full[st], kb * 64, u.g, vrow);
+                tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128, &map_v,
+                            &bars.v_full[st], kb * 64, u.g, vrow);
+            } else {
+              for (int hb = 0; hb < BK / 64; ++hb) {
+                const int32_t vrow = kv_tensor_row((n - 1) * BK + hb * 64, u.b, int32_t(prm.S),
+                                                   int32_t(prm.C), prm.B, prm.D, prm.kv_shard_major);
+                for (int kb = 0; kb < KB; ++kb)
+                  tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
+                              &map_v, &bars.v_full[st], kb * 64, u.g, vrow);
+              }
             }
             ++v_fills[st];
           }

@@ -43,25 +43,36 @@ __global__ void __launch_bounds__(256) zsa_merge_kernel(const __grid_constant__ 
 #pragma unroll
     for (int t = 0; t < 8; ++t) acc[t] = 0.f;
     if (live) {
-      for (int i = 0; i < a.n; ++i) {
-        const float li = a.lse[i][lidx];
-        if (li == -INFINITY) continue;         // an empty key set adds nothing
-        if (li > m) {                          // rescale what was summed against the old max
-          const float c = expf(m - li);        // m = -inf at the first live part: c = 0
-          l *= c;
-#pragma unroll
-          for (int t = 0; t < 8; ++t) acc[t] *= c;
-          m = li;
-        }
-        const float w = expf(li - m);
-        l += w;
-        const uint4 x = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const __nv_bfloat16*>(a.o[i]) + pair * HD)[sub];
-        const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+      // parts in groups of four: every load of a group is issued before any arithmetic,
+      // so their latencies overlap instead of chaining part after part
+      for (int i0 = 0; i0 < a.n; i0 += 4) {
+        float li[4];
+        uint4 x[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          acc[2 * t] = fmaf(w, __uint_as_float(xs[t] << 16), acc[2 * t]);
-          acc[2 * t + 1] = fmaf(w, __uint_as_float(xs[t] & 0xFFFF0000u), acc[2 * t + 1]);
+          const int i = i0 + t < a.n ? i0 + t : i0;
+          li[t] = i0 + t < a.n ? a.lse[i][lidx] : -INFINITY;
+          x[t] = reinterpret_cast<const uint4*>(
+              reinterpret_cast<const __nv_bfloat16*>(a.o[i]) + pair * HD)[sub];
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          if (li[t] == -INFINITY) continue;      // an empty key set (or no part) adds nothing
+          if (li[t] > m) {                       // rescale what was summed against the old max
+            const float c = expf(m - li[t]);     // m = -inf at the first live part: c = 0
+            l *= c;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] *= c;
+            m = li[t];
+          }
+          const float w = expf(li[t] - m);
+          l += w;
+          const uint32_t xs[4] = {x[t].x, x[t].y, x[t].z, x[t].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] = fmaf(w, __uint_as_float(xs[e] << 16), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(w, __uint_as_float(xs[e] & 0xFFFF0000u), acc[2 * e + 1]);
+          }
         }
       }
     }

@@ -25,16 +25,18 @@ ZSA_HD int64_t zigzag_row(int64_t C, int32_t D, int64_t p) {
 
 // Row of a K / V tensor ([rows][Hkv][d]) holding position p of batch b: b*S + p in
 // position order, or the zigzag owner's row (r*B + b)*2C + j in the shard-major order
-// (the all-gather of every shard's own rows).  A 64-key box starting at a multiple of
-// 64 lies inside one zigzag chunk (C % 64 == 0), so its rows are contiguous either way.
-ZSA_HD int32_t kv_tensor_row(int64_t p, int32_t b, int64_t S, int32_t B, int32_t D,
+// (the all-gather of every shard's own rows).  C = S/(2D) is passed in (no division by
+// a 64-bit value on the device); positions and rows fit in 32 bits (B*S < 2^31).  A
+// 64-key box starting at a multiple of 64 lies inside one zigzag chunk (C % 64 == 0),
+// so its rows are contiguous either way.
+ZSA_HD int32_t kv_tensor_row(int32_t p, int32_t b, int32_t S, int32_t C, int32_t B, int32_t D,
                              int32_t shard_major) {
-  if (!shard_major) return int32_t(int64_t(b) * S + p);
-  const int64_t C = S / (2 * int64_t(D));
-  const int64_t c = p / C, o = p % C;
-  const int64_t r = c < D ? c : 2 * D - 1 - c;
-  const int64_t j = c < D ? o : C + o;
-  return int32_t((r * B + b) * 2 * C + j);
+  if (!shard_major) return b * S + p;
+  const uint32_t c = uint32_t(p) / uint32_t(C);
+  const int32_t o = p - int32_t(c) * C;
+  const int32_t r = int32_t(c) < D ? int32_t(c) : 2 * D - 1 - int32_t(c);
+  const int32_t j = int32_t(c) < D ? o : C + o;
+  return (r * B + b) * 2 * C + j;
 }
 
 // Device-side record of one forward work unit (32 bytes).
