@@ -17,7 +17,10 @@
 // streams [128 m][64 k] tiles of X (K-major) and [64 k][128 n] tiles of W_s (two 64-wide
 // n boxes, MN-major) through a 6-stage ring; one thread issues tcgen05.mma (M = N = 128,
 // K = 16) into one of two TMEM accumulators; 4 epilogue warps (thread = output row)
-// drain the other accumulator meanwhile.  Every wait is bounded.
+// drain the other accumulator meanwhile.  fp32-accumulate chunks leave by TMA bulk
+// reduce-add (each warp stages its [32 rows][32 columns] in a double-buffered,
+// 128B-swizzled box), so the accumulator is never read back by the SM; bf16 chunks are
+// stored directly.  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "zsa_kernels.h"
@@ -33,12 +36,19 @@ struct GemmCfg {
   static constexpr int A_BYTES = BM * BK * 2;     // 16 KB
   static constexpr int B_BYTES = BK * BN * 2;     // 16 KB: [2 n blocks][64 k][128 B]
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int STG_BYTES = 4 * 2 * 32 * 128;   // 4 warps x 2 boxes of [32 rows][32 fp32]
+  static constexpr int SMEM_STG = STAGES * STAGE_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_STG + STG_BYTES;
   static constexpr int WARP_LOAD = 4;
   static constexpr int WARP_MMA = 5;
   static constexpr int NTHREADS = 6 * 32;
   static constexpr uint32_t TM_COLS = 256;        // two 128-column accumulators
   static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
+};
+
+// Tensor maps of the fp32-accumulate segments ([T][cols] fp32, [32 rows][32 cols] boxes).
+struct SegMaps {
+  CUtensorMap m[kProjMaxSegs];
 };
 
 struct GemmParams {
@@ -58,7 +68,8 @@ struct GemmBars {
 
 __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
     zsa_proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
-                         const __grid_constant__ CUtensorMap map_w, const GemmParams prm) {
+                         const __grid_constant__ CUtensorMap map_w,
+                         const __grid_constant__ SegMaps seg_maps, const GemmParams prm) {
   using Cfg = GemmCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -155,7 +166,8 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
     // epilogue: thread = output row; 32-column chunks go to their segment
     const uint32_t lane_addr = uint32_t(warp * 32) << 16;
     const int row = warp * 32 + lane;
-    uint32_t tile_it = 0;
+    uint8_t* stg = smem + Cfg::SMEM_STG + warp * (2 * 32 * 128);   // this warp's two boxes
+    uint32_t tile_it = 0, n_red = 0;
     bool ok = true;
     for (int32_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tile_it) {
       const int acc = int(tile_it & 1);
@@ -172,23 +184,30 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
         tmem_ld32(tmem + uint32_t(acc * Cfg::BN + c * 32) + lane_addr, v);
         tmem_ld_wait();
         int64_t col = n0 + c * 32;
-        if (!row_in || col >= prm.N) continue;       // past the output's edge
+        if (col >= prm.N) continue;                  // past the output's edge
         int si = 0;
         while (si + 1 < prm.n_segs && col >= prm.segs[si].col_end) ++si;
         const ProjSegment& sg = prm.segs[si];
         const int64_t oc = col - sg.col_begin;
         if (sg.fp32_accumulate) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(sg.out) + m * sg.ld + oc);
+          // stage [32 rows][32 fp32] (row = lane, 128-byte rows, 128-byte swizzle) and
+          // reduce-add it; the box's other buffer may still be read by the previous reduce
+          uint8_t* box = stg + (n_red & 1) * (32 * 128);
+          if (lane == 0) bulk_wait_group_read1();
+          __syncwarp();
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            float4 y = dst[q4];
-            y.x += __uint_as_float(v[4 * q4]);
-            y.y += __uint_as_float(v[4 * q4 + 1]);
-            y.z += __uint_as_float(v[4 * q4 + 2]);
-            y.w += __uint_as_float(v[4 * q4 + 3]);
-            dst[q4] = y;
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<uint4*>(box + sw128_offset(uint32_t(lane), uint32_t(q4))) =
+                make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&seg_maps.m[si], box, int32_t(oc),
+                              int32_t(int64_t(t % prm.mt) * Cfg::BM + warp * 32), 0);
+            bulk_commit_group();
           }
-        } else {
+          ++n_red;
+        } else if (row_in) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(sg.out) + m * sg.ld + oc);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
@@ -202,6 +221,8 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty[acc]);
     }
+    if (lane == 0) bulk_wait_group0();        // every reduce-add performed before exit
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -226,6 +247,16 @@ int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
     const uint32_t box[3] = {64, uint32_t(Cfg::BK), 1};
     if (!make_map_bf16_sw128(&mw, a.w, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
+  SegMaps sm;
+  for (int i = 0; i < a.n_segs; ++i) {
+    if (!a.segs[i].fp32_accumulate) continue;
+    const uint64_t cols = uint64_t(a.segs[i].col_end - a.segs[i].col_begin);
+    const uint64_t dims[3] = {cols, uint64_t(a.T), 1};
+    const uint64_t strides[2] = {uint64_t(a.segs[i].ld) * 4, uint64_t(a.segs[i].ld) * 4 * uint64_t(a.T)};
+    const uint32_t box[3] = {32, 32, 1};
+    if (!make_map_f32_sw128(&sm.m[i], a.segs[i].out, 3, dims, strides, box))
+      return int(cudaErrorInvalidValue);
+  }
   GemmParams p;
   p.T = a.T; p.N = a.N; p.K = a.K;
   p.mt = int32_t((a.T + Cfg::BM - 1) / Cfg::BM);
@@ -245,7 +276,7 @@ int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
   if (grid <= 0) return int(cudaSuccess);
   const TraceEvents tr = trace_events(5);
   if (tr.begin) cudaEventRecord(tr.begin, stream);
-  zsa_proj_gemm_kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mx, mw, p);
+  zsa_proj_gemm_kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mx, mw, sm, p);
   const cudaError_t err = cudaGetLastError();
   if (tr.end) cudaEventRecord(tr.end, stream);
   return int(err);
