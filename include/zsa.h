@@ -185,8 +185,9 @@ ZSA_API int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* 
  *   lse_parts : HOST array of n_parts device pointers, fp32 [shards][B][Hq][2C]
  *   o, lse    : device outputs in the same layouts; they may alias one of the parts (a
  *               running merge in place)
- * Pointers 16-byte aligned.  Asynchronous on cuda_stream; HBM-bound (reads n_parts *
- * (2d + 4) bytes and writes 2d + 4 per (row, head)). */
+ * Pointers 16-byte aligned; rows * Hq * d < 2^31 (ZSA_ERR_SHAPE otherwise).  Asynchronous
+ * on cuda_stream; HBM-bound (reads n_parts * (2d + 4) bytes and writes 2d + 4 per
+ * (row, head)). */
 ZSA_API int zsa_attn_merge(const zsa_problem* problem, int32_t n_parts, const void* const* o_parts,
                            const float* const* lse_parts, void* o, float* lse,
                            void* cuda_stream);

@@ -350,6 +350,7 @@ int zsa_attn_merge(const zsa_problem* problem, int32_t n_parts, const void* cons
   if (rc) return rc;
   if (n_parts < 1 || n_parts > ZSA_MERGE_MAX_PARTS || !o_parts || !lse_parts || !o || !lse)
     return ZSA_ERR_INVALID;
+  if (local_rows(problem) * problem->Hq * problem->d >= (int64_t(1) << 31)) return ZSA_ERR_SHAPE;
   zsa::MergeArgs a;
   for (int i = 0; i < n_parts; ++i) {
     if (!o_parts[i] || !lse_parts[i] || !aligned16(o_parts[i]) || !aligned16(lse_parts[i]))

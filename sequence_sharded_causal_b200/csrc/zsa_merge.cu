@@ -25,19 +25,23 @@ namespace zsa {
 namespace {
 
 template <int HD>
+// Index arithmetic is 32-bit (the launcher checks that rows * Hq * d < 2^31): 64-bit
+// divisions per (row, head) would make this HBM-bound kernel issue-bound.
 __global__ void __launch_bounds__(256) zsa_merge_kernel(const __grid_constant__ MergeArgs a,
-                                                        int64_t n_pairs, int64_t twoC) {
-  constexpr int LPP = HD / 8;                 // lanes per (row, head), 16 bytes each
-  const int lane = int(threadIdx.x & 31);
-  const int sub = lane % LPP;
-  const int64_t warp_global = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-  const int64_t n_warps = int64_t(gridDim.x) * blockDim.x / 32;
-  for (int64_t base = warp_global * (32 / LPP); base < n_pairs; base += n_warps * (32 / LPP)) {
-    const int64_t pair = base + lane / LPP;   // (row, head) in the O layout's order
+                                                        uint32_t n_pairs, uint32_t twoC) {
+  constexpr uint32_t LPP = HD / 8;            // lanes per (row, head), 16 bytes each
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t sub = lane % LPP;
+  const uint32_t Hq = uint32_t(a.Hq);
+  const uint32_t warp_global = (blockIdx.x * blockDim.x + threadIdx.x) / 32u;
+  const uint32_t n_warps = gridDim.x * blockDim.x / 32u;
+  for (uint32_t base = warp_global * (32u / LPP); base < n_pairs; base += n_warps * (32u / LPP)) {
+    const uint32_t pair = base + lane / LPP;  // (row, head) in the O layout's order
     const bool live = pair < n_pairs;
-    const int64_t row = live ? pair / a.Hq : 0;
-    const int32_t h = live ? int32_t(pair % a.Hq) : 0;
-    const int64_t lidx = ((row / twoC) * a.Hq + h) * twoC + row % twoC;   // lse layout
+    const uint32_t row = live ? pair / Hq : 0u;
+    const uint32_t h = live ? pair - row * Hq : 0u;
+    const uint32_t rb = row / twoC;
+    const uint32_t lidx = (rb * Hq + h) * twoC + (row - rb * twoC);   // lse layout
     float m = -INFINITY, l = 0.f;
     float acc[8];
 #pragma unroll
@@ -53,7 +57,7 @@ __global__ void __launch_bounds__(256) zsa_merge_kernel(const __grid_constant__ 
           const int i = i0 + t < a.n ? i0 + t : i0;
           li[t] = i0 + t < a.n ? a.lse[i][lidx] : -INFINITY;
           x[t] = reinterpret_cast<const uint4*>(
-              reinterpret_cast<const __nv_bfloat16*>(a.o[i]) + pair * HD)[sub];
+              reinterpret_cast<const __nv_bfloat16*>(a.o[i]) + size_t(pair) * HD)[sub];
         }
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(256) zsa_merge_kernel(const __grid_constant__ 
       y.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
       y.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
       y.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-      reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o_out) + pair * HD)[sub] = y;
+      reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o_out) + size_t(pair) * HD)[sub] = y;
       if (sub == 0) a.lse_out[lidx] = empty ? -INFINITY : m + logf(l);
     }
   }
@@ -104,7 +108,7 @@ int launch_merge_hd(const MergeArgs& a, cudaStream_t stream) {
   if (blocks < 1) return int(cudaSuccess);
   const TraceEvents tr = trace_events(4);
   if (tr.begin) cudaEventRecord(tr.begin, stream);
-  zsa_merge_kernel<HD><<<int(blocks), 256, 0, stream>>>(a, n_pairs, twoC);
+  zsa_merge_kernel<HD><<<int(blocks), 256, 0, stream>>>(a, uint32_t(n_pairs), uint32_t(twoC));
   const cudaError_t e = cudaGetLastError();
   if (tr.end) cudaEventRecord(tr.end, stream);
   return int(e);
