@@ -49,8 +49,14 @@ CONFIGS = {
 # targets (S >= 32K) apply.
 DEFAULT_CONFIG = "long"
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of
-# the current kernel (profiles/); configurations without a capture report null.
-MEASURED_TRAFFIC = {}
+# the current kernel at the configuration's full size (dram__bytes_read.sum +
+# dram__bytes_write.sum, a one-pass capture; profiles/dram_traffic_bwd_main.md);
+# configurations without a capture report null.
+MEASURED_TRAFFIC = {
+    ("long", "zsa_bwd_wide_kernel"): 18.71e9 + 10.49e9,
+    ("8b_gqa", "zsa_bwd_wide_kernel"): 1.954867e9 + 1.042157e9,
+    ("wide_gqa", "zsa_bwd_pair_kernel"): 38.77e9 + 22.84e9,
+}
 # Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
 CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
 
@@ -351,7 +357,7 @@ def run_zsa(args, c, name):
     main_tf = bf / world / (kms[2] * 1e-3) / 1e12
     # dominant kernel by time: forward kernel or backward main kernel
     if kms[2] >= kms[0]:
-        dom, dom_tf = ("zsa_bwd_wide_kernel" if d <= 128 else "zsa_bwd_kernel"), main_tf
+        dom, dom_tf = ("zsa_bwd_wide_kernel" if d <= 128 else "zsa_bwd_pair_kernel"), main_tf
     else:
         dom, dom_tf = "zsa_fwd_kernel", fwd_tf
     traffic = MEASURED_TRAFFIC.get((name, dom))
@@ -417,6 +423,80 @@ def _time_events(fn, steps, warmup, dev):
     return e0.elapsed_time(e1) / steps
 
 
+def _component_ring(args, c, zsa, dev, g, peak, hbm, peak_src):
+    import torch
+    B, S, Hq, Hkv, d, D = (c[k] for k in ("B", "S", "Hq", "Hkv", "d", "D"))
+    bf = torch.bfloat16
+    C = S // (2 * D)
+    ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    if args.component == "permute":
+        q = torch.randn((B, S, Hq, d), generator=g, device=dev).to(bf)
+        k = torch.randn((B, S, Hkv, d), generator=g, device=dev).to(bf)
+        v = torch.randn((B, S, Hkv, d), generator=g, device=dev).to(bf)
+        qs = torch.empty((D, B, S // D, Hq, d), dtype=bf, device=dev)
+        ks = torch.empty((D, B, S // D, Hkv, d), dtype=bf, device=dev)
+        vs = torch.empty_like(ks)
+
+        def step():
+            zsa.to_shard_major(q, D, out=qs)
+            zsa.to_shard_major(k, D, out=ks)
+            zsa.to_shard_major(v, D, out=vs)
+        zsa.zsa_trace_events(zsa.ZSA_TRACE_PERMUTE, ev[0], ev[1])
+        ms = _time_events(step, args.steps, args.warmup, dev)
+        zsa.zsa_trace_events(zsa.ZSA_TRACE_PERMUTE, None, None)
+        kms = ev[0].elapsed_time(ev[1])                 # the last V copy alone
+        nbytes = 2 * 2 * B * S * (Hq + 2 * Hkv) * d
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        k_gbs = 2 * 2 * B * S * Hkv * d / (kms * 1e-3) / 1e9
+        return {"metric": "K5 natural -> zigzag shard-major permute GB/s at 1 B200", "value": gbs,
+                "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": c["desc"] + ", Q, K and V to shard-major order"},
+                "roofline": {"kernel": "zsa_permute_kernel", "bound": "hbm", "achieved": gbs,
+                             "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                             "peak_source": f"{peak_src} copy bandwidth", "traffic": None,
+                             "last_launch_gbs": k_gbs},
+                "gpu_launches": 3 * args.steps}
+    q = torch.randn((D, B, S // D, Hq, d), generator=g, device=dev).to(bf)
+    k = torch.randn((B, S, Hkv, d), generator=g, device=dev).to(bf)
+    v = torch.randn((B, S, Hkv, d), generator=g, device=dev).to(bf)
+    o, lse = torch.empty_like(q), torch.empty((D, B, Hq, S // D), device=dev)
+    o_p, lse_p = torch.empty_like(q), torch.empty_like(lse)
+    problem = zsa.make_problem(B, S, Hq, Hkv, d, D)
+    ws = torch.empty(zsa.zsa_workspace_bytes(problem, 0), dtype=torch.uint8, device=dev)
+    # the ring order of rank 0: its own chunks first
+    chunks = []
+    for s_ in range(D):
+        chunks += [s_, 2 * D - 1 - s_]
+
+    def step():
+        for i, ch in enumerate(chunks):
+            dst = (o, lse) if i == 0 else (o_p, lse_p)
+            zsa.attn_fwd_block(q, k, v, D, ch * C, (ch + 1) * C, rows_per_batch=S,
+                               row_offset=ch * C, workspace=ws, out=dst)
+            if i > 0:
+                zsa.zsa_attn_merge(problem, [o, o_p], [lse, lse_p], o, lse)
+    zsa.zsa_trace_events(zsa.ZSA_TRACE_MERGE, ev[0], ev[1])
+    ms = _time_events(step, args.steps, args.warmup, dev)
+    zsa.zsa_trace_events(zsa.ZSA_TRACE_MERGE, None, None)
+    if zsa.zsa_device_status(ws) != zsa.ZSA_OK:
+        raise RuntimeError("key-block forward reported a timeout")
+    flops = fwd_flops(c)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"metric": "ring-attention forward (key blocks + running merge) TFLOP/s at 1 B200",
+            "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{c['desc']}: {2 * D} key blocks of C={C} positions, "
+                                   f"{2 * D - 1} in-place merges"},
+            "roofline": {"kernel": "zsa_fwd_kernel (key-block)", "bound": "tensor",
+                         "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "peak_source": f"{peak_src} bf16 burst", "traffic": None,
+                         "last_merge_ms": ev[0].elapsed_time(ev[1])},
+            "gpu_launches": (4 * D - 1) * args.steps}
+
+
 def run_component(args, c, name):
     """One JSON line for a NEXT-row kernel on one GPU, at the configuration's sizes.
 
@@ -426,6 +506,11 @@ def run_component(args, c, name):
     tsp_projection: one rank's D projection steps of the TSP attention layer (QKV from
       the packed shards, then the output projection's fp32 partials), the rank's tokens
       T = B*S/D, hidden = the model's width; the broadcast is local on one GPU.
+    permute: K5, natural -> zigzag shard-major copies of Q, K and V (HBM-bound: each
+      byte read and written once).
+    ring_forward: the forward as ring attention computes it, on one GPU: every shard's
+      queries against one zigzag chunk of K/V at a time (2D key-block launches), each
+      partial merged into the running (O, lse) in place; TFLOP/s of the causal FLOPs.
     """
     import torch
     import sequence_sharded_causal_b200 as zsa
@@ -434,7 +519,9 @@ def run_component(args, c, name):
     B, S, Hq, Hkv, d, D = (c[k] for k in ("B", "S", "Hq", "Hkv", "d", "D"))
     peak, peak_sus, hbm, peak_src = load_peaks()
     g = torch.Generator(device=dev).manual_seed(c["seed"])
-    if args.component == "merge":
+    if args.component in ("permute", "ring_forward"):
+        line = _component_ring(args, c, zsa, dev, g, peak, hbm, peak_src)
+    elif args.component == "merge":
         problem = zsa.make_problem(B, S, Hq, Hkv, d, D)
         shp, lshp = (D, B, S // D, Hq, d), (D, B, Hq, S // D)
         o = torch.randn(shp, generator=g, device=dev).to(torch.bfloat16)
@@ -516,9 +603,11 @@ def main():
     ap.add_argument("--impl", default="zsa", choices=("zsa", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--component", default="attention",
-                    choices=("attention", "merge", "tsp_projection"),
-                    help="attention: the hot path (default); merge / tsp_projection: the "
-                         "ring-attention merge or the TSP projection schedule on one GPU")
+                    choices=("attention", "merge", "tsp_projection", "permute", "ring_forward"),
+                    help="attention: the hot path (default); merge / tsp_projection / "
+                         "permute / ring_forward: the ring-attention merge, the TSP "
+                         "projection schedule, the K5 permute or a ring-attention forward "
+                         "on one GPU")
     ap.add_argument("--seq", type=int, default=0,
                     help="run the configuration's heads, d and D at this sequence length "
                          "(profiling captures of a smaller case); 0 = the configuration's S")

@@ -192,6 +192,57 @@ ZSA_API int zsa_attn_merge(const zsa_problem* problem, int32_t n_parts, const vo
                            const float* const* lse_parts, void* o, float* lse,
                            void* cuda_stream);
 
+/* K5: copy a tensor of one bf16 row of heads*d values per position between the natural
+ * order [B][S][heads][d] and the zigzag shard-major order [shards][B][2C][heads][d] of the
+ * problem's shard range (all D by default): shard r holds chunk r, then chunk 2D-1-r, of
+ * C = S/(2D) positions ("Folding Tensor and Sequence Parallelism" summary, section 2,
+ * attention layer: the zigzag partition of the sequence).  For callers whose Q, O, dO or
+ * K/V are in position order; the attention calls themselves need no such pass
+ * (ZSA_KV_SHARD_MAJOR reads an all-gather's output as it lands).
+ *   heads          : Hq for Q / O / dO / dQ, Hkv for K / V / dK / dV (any value >= 1)
+ *   to_shard_major : 1: src natural -> dst shard-major; 0: src shard-major -> dst natural.
+ *                    With a shard range, natural -> shard-major reads only the range's
+ *                    chunks, and shard-major -> natural writes only those (the other rows
+ *                    of dst are left as they are).
+ *   src, dst       : device pointers, 16-byte aligned, not overlapping.
+ * Uses the problem's B, S, D, d and shard range (d a multiple of 8; Hq, Hkv, the scale and
+ * kv_layout are checked as everywhere but not used).  ZSA_ERR_SHAPE when 2 * shards * B >
+ * 65535.  Asynchronous on cuda_stream; HBM-bound (reads and writes each byte once). */
+ZSA_API int zsa_permute(const zsa_problem* problem, int32_t heads, int32_t to_shard_major,
+                        const void* src, void* dst, void* cuda_stream);
+
+/* A block of keys for zsa_attn_fwd_block: the positions [key_lo, key_hi) of the
+ * sequence (0 <= key_lo <= key_hi <= S, any values), held in K/V tensors
+ * [rows][Hkv][d] bf16 with the key at position p of batch b in row
+ *   b * rows_per_batch + row_offset + (p - key_lo).
+ * E.g. one zigzag chunk c of a natural [B][S][Hkv][d] buffer: rows_per_batch = S,
+ * row_offset = c*C; the first chunk of a received shard block [B][2C][Hkv][d]:
+ * rows_per_batch = 2C, row_offset = 0 (its second chunk: row_offset = C).
+ * rows, rows_per_batch and row_offset are below 2^31, and every row the block names lies
+ * inside the tensor: (B-1)*rows_per_batch + row_offset + (key_hi - key_lo) <= rows, with
+ * rows_per_batch >= key_hi - key_lo when B > 1. */
+typedef struct {
+  int64_t key_lo, key_hi;
+  int64_t rows_per_batch;
+  int64_t row_offset;
+  int64_t rows;
+} zsa_key_block;
+
+/* Forward restricted to one block of keys: the partial result one ring-attention step
+ * computes ("AutoSP" summary, sections 1 and 4, ring attention as the sequence-parallel
+ * baseline: each rank's queries meet the K/V blocks one at a time).  For every query
+ * row of the problem's shard range and q head: the causal softmax attention over the
+ * keys of the block only (the mask on global positions as in zsa_attn_fwd), written as
+ * o (bf16, Q layout) and lse (fp32 [shards][B][Hq][2C]) exactly as zsa_attn_fwd writes
+ * them.  A row that sees no key of the block gets o = 0 and lse = -inf, the empty part
+ * zsa_attn_merge skips; merging the results of blocks that tile [0, S) gives
+ * zsa_attn_fwd's.  problem->kv_layout is not used (the block describes K/V).  Workspace
+ * as zsa_attn_fwd's (zsa_workspace_bytes pass 0); pointers 16-byte aligned; errors as
+ * zsa_attn_fwd, plus ZSA_ERR_INVALID for a block outside the bounds above. */
+ZSA_API int zsa_attn_fwd_block(const zsa_problem* problem, const zsa_key_block* block,
+                               const void* q, const void* k, const void* v, void* o, float* lse,
+                               void* workspace, size_t ws_bytes, void* cuda_stream);
+
 /* One run of output columns of a TSP projection step (zsa_tsp_project). */
 typedef struct {
   void* out;                 /* device: element (0, 0) of this run's output */
@@ -273,10 +324,11 @@ ZSA_API int zsa_debug_inject_stall(int enable);
  * kernel alone with cudaEventElapsedTime.  which: ZSA_TRACE_FWD (forward kernel),
  * ZSA_TRACE_BWD_PRE (Delta preprocess), ZSA_TRACE_BWD_MAIN (backward main kernel),
  * ZSA_TRACE_BWD_DQ (dQ conversion), ZSA_TRACE_MERGE (partial-result merge),
- * ZSA_TRACE_PROJ (TSP projection GEMM).  Pass NULL events to stop tracing that kernel. */
+ * ZSA_TRACE_PROJ (TSP projection GEMM), ZSA_TRACE_PERMUTE (K5 permute).  Pass NULL events
+ * to stop tracing that kernel. */
 enum {
   ZSA_TRACE_FWD = 0, ZSA_TRACE_BWD_PRE = 1, ZSA_TRACE_BWD_MAIN = 2, ZSA_TRACE_BWD_DQ = 3,
-  ZSA_TRACE_MERGE = 4, ZSA_TRACE_PROJ = 5
+  ZSA_TRACE_MERGE = 4, ZSA_TRACE_PROJ = 5, ZSA_TRACE_PERMUTE = 6
 };
 ZSA_API int zsa_trace_events(int which, void* begin_event, void* end_event);
 

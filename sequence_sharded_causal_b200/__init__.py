@@ -36,10 +36,10 @@ ZSA_KV_SHARD_MAJOR = 1
 EXPORTED = ("zsa_partition", "zsa_workspace_bytes", "zsa_attn_fwd", "zsa_attn_bwd",
             "zsa_device_status", "zsa_set_wait_limit_ns", "zsa_debug_inject_stall",
             "zsa_trace_events", "zsa_attn_merge", "zsa_tsp_project", "zsa_attn_bwd_noalloc",
-            "zsa_noalloc_status", "zsa_status_string")
+            "zsa_noalloc_status", "zsa_attn_fwd_block", "zsa_permute", "zsa_status_string")
 ZSA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 (ZSA_TRACE_FWD, ZSA_TRACE_BWD_PRE, ZSA_TRACE_BWD_MAIN, ZSA_TRACE_BWD_DQ, ZSA_TRACE_MERGE,
- ZSA_TRACE_PROJ) = range(6)
+ ZSA_TRACE_PROJ, ZSA_TRACE_PERMUTE) = range(7)
 ZSA_PROJ_MAX_SEGMENTS = 8
 ZSA_MERGE_MAX_PARTS = 32
 
@@ -64,6 +64,11 @@ class zsa_work(ctypes.Structure):
 class zsa_proj_segment(ctypes.Structure):
     _fields_ = [("out", ctypes.c_void_p), ("ld", ctypes.c_int64), ("cols", ctypes.c_int32),
                 ("fp32_accumulate", ctypes.c_int32)]
+
+
+class zsa_key_block(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("key_lo", "key_hi", "rows_per_batch", "row_offset",
+                                              "rows")]
 
 
 class ZsaError(RuntimeError):
@@ -99,6 +104,9 @@ def lib():
         L.zsa_tsp_project.argtypes = [i64, i64, i64, vp, i64, vp, i64, vp, ctypes.c_int32, vp, vp]
         L.zsa_attn_bwd_noalloc.argtypes = [P(zsa_problem)] + [vp] * 10
         L.zsa_noalloc_status.argtypes = [vp]
+        L.zsa_permute.argtypes = [P(zsa_problem), ctypes.c_int32, ctypes.c_int32, vp, vp, vp]
+        L.zsa_attn_fwd_block.argtypes = [P(zsa_problem), P(zsa_key_block), vp, vp, vp, vp, vp, vp,
+                                         ctypes.c_size_t, vp]
         L.zsa_status_string.argtypes = [ctypes.c_int]
         L.zsa_status_string.restype = ctypes.c_char_p
         for name in EXPORTED[:-1]:
@@ -182,6 +190,19 @@ def zsa_attn_fwd(problem, q, k, v, o, lse, workspace, ws_bytes=None, stream=None
     _check(lib().zsa_attn_fwd(ctypes.byref(problem), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                               _ptr(lse), _ptr(workspace), int(ws_bytes), _stream(stream)),
            "zsa_attn_fwd")
+
+
+def zsa_attn_fwd_block(problem, block, q, k, v, o, lse, workspace, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().zsa_attn_fwd_block(ctypes.byref(problem), ctypes.byref(block), _ptr(q), _ptr(k),
+                                    _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace), int(ws_bytes),
+                                    _stream(stream)), "zsa_attn_fwd_block")
+
+
+def zsa_permute(problem, heads, to_shard_major, src, dst, stream=None):
+    _check(lib().zsa_permute(ctypes.byref(problem), int(heads), int(to_shard_major), _ptr(src),
+                             _ptr(dst), _stream(stream)), "zsa_permute")
 
 
 def zsa_attn_bwd(problem, q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes=None,
@@ -315,6 +336,74 @@ def attn_fwd(q, k, v, D, causal=True, scale=None, workspace=None, kv_layout=ZSA_
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     zsa_attn_fwd(problem, q, k, v, o, lse, workspace)
     return o, lse
+
+
+def attn_fwd_block(q, k, v, D, key_lo, key_hi, rows_per_batch=None, row_offset=0, causal=True,
+                   scale=None, workspace=None, shard_begin=0, shard_count=0, out=None):
+    """Partial O, lse over the keys at positions [key_lo, key_hi) only (one ring step).
+
+    k, v: contiguous (..., Hkv, d) tensors whose leading dims flatten to the K/V rows; the
+    key at position p of batch b is row b * rows_per_batch + row_offset + p - key_lo
+    (rows_per_batch defaults to key_hi - key_lo: a [B][key_hi - key_lo][Hkv][d] block).
+    out: optional (o, lse) to write into."""
+    import torch
+    ns, B, twoC, Hq, d = q.shape
+    Hkv = k.shape[-2]
+    if shard_count == 0 and ns != D:
+        raise ValueError(f"q holds {ns} shards; pass shard_begin / shard_count for a subset of D={D}")
+    problem = make_problem(B, D * twoC, Hq, Hkv, d, D, causal, scale, ZSA_KV_NATURAL, shard_begin,
+                           shard_count)
+    qs, _, ls = _shapes(problem)
+    _check_tensor(q, qs, torch.bfloat16, "q")
+    rows = k.numel() // (Hkv * d)
+    _check_tensor(k, tuple(k.shape), torch.bfloat16, "k")
+    _check_tensor(v, tuple(k.shape), torch.bfloat16, "v")
+    if k.shape[-1] != d:
+        raise ValueError(f"k head dim {k.shape[-1]} != q head dim {d}")
+    block = zsa_key_block(int(key_lo), int(key_hi),
+                          int(key_hi - key_lo if rows_per_batch is None else rows_per_batch),
+                          int(row_offset), int(rows))
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(ls, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+        _check_tensor(o, qs, torch.bfloat16, "o")
+        _check_tensor(lse, ls, torch.float32, "lse")
+    nbytes = zsa_workspace_bytes(problem, 0)
+    if workspace is None or workspace.numel() * workspace.element_size() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    zsa_attn_fwd_block(problem, block, q, k, v, o, lse, workspace)
+    return o, lse
+
+
+def to_shard_major(x, D, shard_begin=0, shard_count=0, out=None):
+    """K5: natural [B][S][H][d] bf16 -> zigzag shard-major [shards][B][2C][H][d]."""
+    import torch
+    B, S, H, d = x.shape
+    ns = shard_count or D
+    problem = make_problem(B, S, H, H, d, D, shard_begin=shard_begin, shard_count=shard_count)
+    _check_tensor(x, (B, S, H, d), torch.bfloat16, "x")
+    if out is None:
+        out = torch.empty((ns, B, S // D, H, d), dtype=torch.bfloat16, device=x.device)
+    _check_tensor(out, (ns, B, S // D, H, d), torch.bfloat16, "out")
+    zsa_permute(problem, H, 1, x, out)
+    return out
+
+
+def from_shard_major(y, D, shard_begin=0, shard_count=0, out=None):
+    """K5: zigzag shard-major [shards][B][2C][H][d] bf16 -> natural [B][S][H][d] (with a
+    shard range, only that range's positions of `out` are written)."""
+    import torch
+    ns, B, twoC, H, d = y.shape
+    S = D * twoC
+    problem = make_problem(B, S, H, H, d, D, shard_begin=shard_begin, shard_count=shard_count)
+    _check_tensor(y, ((shard_count or D), B, twoC, H, d), torch.bfloat16, "y")
+    if out is None:
+        out = torch.empty((B, S, H, d), dtype=torch.bfloat16, device=y.device)
+    _check_tensor(out, (B, S, H, d), torch.bfloat16, "out")
+    zsa_permute(problem, H, 0, y, out)
+    return out
 
 
 def attn_bwd(q, k, v, o, lse, do, D, causal=True, scale=None, workspace=None,

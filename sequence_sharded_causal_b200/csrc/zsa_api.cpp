@@ -27,7 +27,7 @@ using zsa::Schedule;
 constexpr size_t kStatusBytes = 256;
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_inject_stall{0};
-constexpr int kTraceKernels = 6;
+constexpr int kTraceKernels = 7;
 std::atomic<void*> g_trace_begin[kTraceKernels];
 std::atomic<void*> g_trace_end[kTraceKernels];
 
@@ -264,8 +264,11 @@ int zsa_workspace_bytes(const zsa_problem* problem, int pass, size_t* bytes_out)
   return ZSA_OK;
 }
 
-int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
-                 void* o, float* lse, void* workspace, size_t ws_bytes, void* cuda_stream) {
+namespace {
+// The forward over all keys (block == nullptr) or over one block of keys.
+int attn_fwd_impl(const zsa_problem* problem, const zsa_key_block* block, const void* q,
+                  const void* k, const void* v, void* o, float* lse, void* workspace,
+                  size_t ws_bytes, void* cuda_stream) {
   int rc = check_device_problem(problem);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse || !workspace) return ZSA_ERR_INVALID;
@@ -302,8 +305,43 @@ int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const
   a.status = reinterpret_cast<int*>(ws);
   a.wait_limit_ns = g_wait_limit_ns.load();
   a.inject_stall = g_inject_stall.load();
+  if (block) {
+    a.key_block = 1;
+    a.key_lo = int32_t(block->key_lo);
+    a.key_hi = int32_t(block->key_hi);
+    a.kv_rows_per_batch = int32_t(block->rows_per_batch);
+    a.kv_row_offset = int32_t(block->row_offset);
+    a.kv_rows = int32_t(block->rows);
+  }
   if (zsa::launch_fwd(a, stream) != int(cudaSuccess)) return ZSA_ERR_CUDA;
   return ZSA_OK;
+}
+
+bool key_block_ok(const zsa_problem* p, const zsa_key_block* kb) {
+  const int64_t lim = int64_t(1) << 31;
+  if (kb->key_lo < 0 || kb->key_hi < kb->key_lo || kb->key_hi > p->S) return false;
+  if (kb->rows <= 0 || kb->rows >= lim || kb->row_offset < 0 || kb->row_offset >= lim ||
+      kb->rows_per_batch < 0 || kb->rows_per_batch >= lim)
+    return false;
+  const int64_t len = kb->key_hi - kb->key_lo;
+  if (p->B > 1 && kb->rows_per_batch < len) return false;
+  return (p->B - 1) * kb->rows_per_batch + kb->row_offset + len <= kb->rows;
+}
+}  // namespace
+
+int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
+                 void* o, float* lse, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return attn_fwd_impl(problem, nullptr, q, k, v, o, lse, workspace, ws_bytes, cuda_stream);
+}
+
+int zsa_attn_fwd_block(const zsa_problem* problem, const zsa_key_block* block, const void* q,
+                       const void* k, const void* v, void* o, float* lse, void* workspace,
+                       size_t ws_bytes, void* cuda_stream) {
+  if (!problem || !block) return ZSA_ERR_INVALID;
+  const int rc = check_problem(problem);
+  if (rc) return rc;
+  if (!key_block_ok(problem, block)) return ZSA_ERR_INVALID;
+  return attn_fwd_impl(problem, block, q, k, v, o, lse, workspace, ws_bytes, cuda_stream);
 }
 
 int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const void* v,
@@ -341,6 +379,40 @@ int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const
   const int e = zsa::launch_bwd(a, stream);
   if (e == int(cudaErrorNotSupported)) return ZSA_ERR_UNSUPPORTED;
   if (e != int(cudaSuccess)) return ZSA_ERR_CUDA;
+  return ZSA_OK;
+}
+
+int zsa_permute(const zsa_problem* problem, int32_t heads, int32_t to_shard_major,
+                const void* src, void* dst, void* cuda_stream) {
+  if (!problem) return ZSA_ERR_INVALID;
+  int rc = check_problem(problem);
+  if (rc) return rc;
+  if (problem->d <= 0 || problem->d % 8 != 0 || heads <= 0) return ZSA_ERR_INVALID;
+  if (to_shard_major != 0 && to_shard_major != 1) return ZSA_ERR_INVALID;
+  if (!src || !dst || !aligned16(src) || !aligned16(dst)) return ZSA_ERR_INVALID;
+  const int64_t C = problem->S / (2 * int64_t(problem->D));
+  const int64_t row_bytes = int64_t(heads) * problem->d * 2;
+  // the two tensors must not overlap (the copy is not ordered)
+  const uintptr_t nat_bytes = uintptr_t(problem->B * problem->S * row_bytes);
+  const uintptr_t smj_bytes = uintptr_t(local_rows(problem) * row_bytes);
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+  const uintptr_t s_bytes = to_shard_major ? nat_bytes : smj_bytes;
+  const uintptr_t d_bytes = to_shard_major ? smj_bytes : nat_bytes;
+  if (s0 < d0 + d_bytes && d0 < s0 + s_bytes) return ZSA_ERR_INVALID;
+  if (2 * int64_t(local_shards(problem)) * problem->B > 65535) return ZSA_ERR_SHAPE;  // grid.y
+  rc = check_sm100();
+  if (rc) return rc;
+  zsa::PermuteArgs a;
+  a.src = src;
+  a.dst = dst;
+  a.chunk_words = C * row_bytes / 16;
+  a.B = int32_t(problem->B);
+  a.D = problem->D;
+  a.shard_begin = problem->shard_begin;
+  a.shard_count = local_shards(problem);
+  a.to_shard_major = to_shard_major;
+  if (zsa::launch_permute(a, static_cast<cudaStream_t>(cuda_stream)) != int(cudaSuccess))
+    return ZSA_ERR_CUDA;
   return ZSA_OK;
 }
 

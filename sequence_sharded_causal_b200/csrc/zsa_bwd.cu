@@ -13,12 +13,12 @@
 // (the single-GPU stand-in for the reduce-scatter back to the owning shards); dQ is
 // summed across key tiles with fp32 reductions into a workspace accumulator.
 //
-// K3 has two builds, chosen by head dim; both use one persistent CTA per SM that
-// claims key-tile units from a global counter in (b, kv head, key tile) order, keep the
-// unit's K and V tiles (128 keys) in shared memory, stream the q slots that see the tile
-// through a 2-stage TMA ring (Q, dO, lse, Delta), and bound every mbarrier wait.
+// K3 has two builds, chosen by head dim.  Both claim 128-key-tile units (b, kv head, key
+// tile) from a global counter in that order, keep the unit's K and V tiles in shared
+// memory, stream the q slots that see the tile through a TMA ring (Q, dO, lse, Delta),
+// send dQ^T through shared memory into TMA bulk reduce-adds, and bound every wait.
 //
-//  zsa_bwd_wide_kernel (d <= 128):
+//  zsa_bwd_wide_kernel (d <= 128, this file): one CTA per key tile;
 //   * 128-row q slots, so all five MMAs of a slot are N = 128; a 128-row slot may
 //     straddle two zigzag chunks, so the 8 compute warps work in two groups of 64
 //     rows, each over contiguous positions;
@@ -27,17 +27,13 @@
 //     warps have read it, dQ^T = K^T dS^T (A = the resident K tile read MN-major, B =
 //     dS^T in shared memory);
 //   * two MMA-issuing threads: one issues S^T and dP^T, the other dV, dK and dQ^T;
-//   * 4 dQ warps read dQ^T out of TMEM and reduce it into the fp32 accumulator.
+//   * 4 dQ warps stage dQ^T in the slot's own Q / dO stage and reduce it into the fp32
+//     accumulator.
 //
-//  zsa_bwd_kernel (d = 256):
-//   * dK + dV of a 128-key tile at d = 256 would fill all of TMEM, so each key tile is
-//     two units, one per 128-wide d chunk; both recompute S^T and dP^T;
-//   * 32-row q slots keep K and V (128 KB) plus the Q/dO ring in shared memory;
-//   * TMEM: dV | dK (the chunk) | S^T x2 | dP^T | dQ^T; dS^T also goes to shared memory
-//     (K-major) as the B operand of dQ^T;
-//   * one MMA-issuing thread; 8 compute warps; 4 dQ warps as above.
+//  zsa_bwd_pair_kernel (d = 256, zsa_bwd_pair.cu): a cluster of two CTAs per key tile,
+//  one holding K and dK, the other V and dV, exchanging P^T and dS^T through
+//  distributed shared memory (dK + dV of the tile alone would fill one SM's TMEM).
 #include <cuda_bf16.h>
-
 
 #include "zsa_bwd_common.cuh"
 #include "zsa_kernels.h"
@@ -252,7 +248,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         unit_ring[slot] = idx;
         mbar_arrive(&bars.unit_full[slot]);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
         if (kv_fills > 0) ok = mbar_wait(&bars.kv_empty, (kv_fills - 1) & 1, wctx);
         if (!ok) break;
         mbar_expect_tx(&bars.kv_full, 2 * Cfg::KV_BYTES);
@@ -335,7 +331,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
         mbar_arrive(&bars.unit_empty[slot]);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
         if (role_a) {
           ok = mbar_wait(&bars.kv_full, kv_ph, wctx);
           kv_ph ^= 1;
@@ -436,7 +432,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
       if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
       SlotWalk w;
       for (bool more = walk_first(prm, u.n, w); more; more = walk_next(prm, u.n, w)) {
         ok = warp_wait_b(&bars.dq_full, dq_ph, wctx);
@@ -507,7 +503,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
       if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
       const int64_t key = int64_t(u.n) * BKV + row;
       SlotWalk w;
       nslots = 0;
@@ -698,7 +694,6 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = a.Hq / a.Hkv; p.D = a.D; p.causal = a.causal;
   p.n_units = int32_t(int64_t(a.B) * a.Hkv * (a.S / BKV));
   p.n_qtiles = int32_t(twoC / BQ);
-  p.n_chunks = 1;
   p.bq = BQ;
   p.n_ktiles = int32_t(a.S / BKV);
   p.kv_shard_major = a.kv_layout;

@@ -21,7 +21,7 @@ struct BwdParams {
   int64_t S, C;
   int32_t B, Hq, Hkv, G, D, causal;
   int32_t n_units, n_qtiles;  // n_qtiles = BQ-row tiles per shard
-  int32_t n_chunks, bq;       // d chunks per key tile, query rows per slot
+  int32_t bq;                 // query rows per slot
   int32_t n_ktiles;           // S / 128
   int32_t kv_shard_major;     // K/V/dK/dV rows in the shard-major zigzag order
   int32_t kv_box;             // rows per K / V TMA box (128, or 64 when C % 128 != 0)
@@ -36,20 +36,18 @@ struct BwdParams {
 
 // One key tile of work.
 struct KvUnit {
-  int32_t n, b, g, c;   // key tile, batch, kv head, d chunk
+  int32_t n, b, g;   // key tile, batch, kv head
 };
 
-// Units are claimed dynamically in the order (b, kv head g, key tile n, d chunk c):
-// CTAs busy at the same time work on one head group, sharing its Q / dO stream and
-// its dQ accumulator rows in L2; within a group n ascends, i.e. the work per unit
-// (the number of q tiles that see key tile n) descends, so each group ends with its
-// shortest units.
-__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int Hkv, int NT, int NC) {
+// Units are claimed dynamically in the order (b, kv head g, key tile n): CTAs busy at
+// the same time work on one head group, sharing its Q / dO stream and its dQ
+// accumulator rows in L2; within a group n ascends, i.e. the work per unit (the number
+// of q tiles that see key tile n) descends, so each group ends with its shortest units.
+__device__ __forceinline__ KvUnit decode_kv_unit(int idx, int Hkv, int NT) {
   KvUnit u;
-  u.c = idx % NC;
-  u.n = (idx / NC) % NT;
-  u.g = (idx / (NC * NT)) % Hkv;
-  u.b = idx / (NC * NT * Hkv);
+  u.n = idx % NT;
+  u.g = (idx / NT) % Hkv;
+  u.b = idx / (NT * Hkv);
   return u;
 }
 

@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
           idx = take_unit(bars, unit_ring, slot, rank);
         }
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
         // the unit's K (CTA 0) or V (CTA 1) tile
         if (t_fills > 0) ok = mbar_wait(&bars.t_empty, (t_fills - 1) & 1, wctx);
         if (!ok) break;
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         if (!ok) break;
         const int idx = take_unit(bars, unit_ring, slot, rank);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
         if (role_a) {
           ok = mbar_wait(&bars.t_full, t_ph, wctx);
           t_ph ^= 1;
@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
         if (idx < 0) break;
-        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+        const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
         SlotWalk w;
         for (bool more = walk_first(prm, u.n, w); more && ok; more = walk_next(prm, u.n, w)) {
           const int32_t h = u.g * prm.G + w.e;
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
         else mbar_arrive_cluster(peer_addr(&bars.unit_empty[slot], 0));
       }
       if (idx < 0) break;
-      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles, 1);
+      const KvUnit u = decode_kv_unit(idx, prm.Hkv, prm.n_ktiles);
       const int64_t key = int64_t(u.n) * BKV + row;
       int nslots = 0;
       SlotWalk w;

@@ -73,10 +73,21 @@ struct FwdParams {
   float* lse;
   int64_t S, C;
   int32_t B, Hq, Hkv, D, causal;
-  int32_t kv_shard_major;  // K/V rows in the shard-major zigzag order instead of position order
-  int32_t shard_begin;     // first shard this launch computes (Q-layout rows are local)
-  int32_t kv_box;          // rows per K / V TMA box: BK when a key tile never straddles a
-                           // zigzag chunk (C % BK == 0), else 64 (C is a multiple of 64)
+  // A key-block launch (KR) reuses the two K/V layout fields for its linear row map.
+  // (The parameter block is kept this small on purpose: at the d <= 128 register budget
+  // a few more words of it made ptxas spill in the softmax warps.)
+  union {
+    int32_t kv_shard_major;  // K/V rows in the shard-major zigzag order instead of position order
+    int32_t kb_rpb;          // KR: K/V rows per batch
+  };
+  int32_t shard_begin;       // first shard this launch computes (Q-layout rows are local)
+  union {
+    int32_t kv_box;          // rows per K / V TMA box: BK when a key tile never straddles a
+                             // zigzag chunk (C % BK == 0), else 64 (C is a multiple of 64)
+    int32_t kb_off;          // KR: K/V row of (batch 0, position key_lo)
+  };
+  int32_t key_lo, key_hi;    // KR: only keys at positions [key_lo, key_hi) count; the key at
+                             // position p of batch b is K/V row b * kb_rpb + kb_off + p - key_lo
   float scale_log2;
   int* status;
   int* counter;       // next unclaimed unit (zeroed before every launch)
@@ -95,13 +106,18 @@ struct FwdBars {
   uint64_t never;  // test hook: no one ever arrives here
 };
 
+// kend[s] counts the slot's key tiles from n0 on: all tiles up to the causal limit
+// (n0 = 0), or, in a key-range launch, those inside [n_lo, n_hi) (n0 = n_lo; a present
+// slot may then have none: its rows see no key of the range).
 struct UnitInfo {
   int32_t r, b, g;
   int32_t tile[2], head[2], kend[2];
-  int32_t nmax;
+  int32_t nmax, n0;
+  uint32_t live;           // bit s: slot s holds a q tile (its kend before any clamp > 0)
 };
 
-__device__ __forceinline__ UnitInfo load_unit(const DevUnit* units, int idx) {
+template <int HD, bool KR>
+__device__ __forceinline__ UnitInfo load_unit(const DevUnit* units, int idx, const FwdParams& prm) {
   const int4* p = reinterpret_cast<const int4*>(units + idx);
   int4 a = __ldg(p), c = __ldg(p + 1);
   UnitInfo u;
@@ -109,8 +125,29 @@ __device__ __forceinline__ UnitInfo load_unit(const DevUnit* units, int idx) {
   u.tile[0] = a.w; u.head[0] = c.x; u.tile[1] = c.y; u.head[1] = c.z;
   u.kend[0] = c.w & 0xFFFF;
   u.kend[1] = (c.w >> 16) & 0xFFFF;
+  u.n0 = 0;
+  u.live = (u.kend[0] > 0 ? 1u : 0u) | (u.kend[1] > 0 ? 2u : 0u);
+  if constexpr (KR) {
+    // the block's key tiles are [n_lo, n_hi)
+    const int32_t n_lo = prm.key_lo / FwdCfg<HD>::BK;
+    const int32_t n_hi = (prm.key_hi + FwdCfg<HD>::BK - 1) / FwdCfg<HD>::BK;
+    u.n0 = n_lo;
+    for (int s = 0; s < 2; ++s) {
+      const int32_t e = u.kend[s] < n_hi ? u.kend[s] : n_hi;
+      u.kend[s] = e > n_lo ? e - n_lo : 0;
+    }
+  }
   u.nmax = u.kend[0] > u.kend[1] ? u.kend[0] : u.kend[1];
   return u;
+}
+
+// K/V tensor row of the key at position p of batch b.  A key-block launch maps positions
+// linearly, so a whole BK tile is one box even where it overhangs the block: rows before
+// the block (a negative coordinate reads zeros) or past it hold keys the mask removes.
+template <bool KR>
+__device__ __forceinline__ int32_t kv_row(const FwdParams& prm, int32_t p, int32_t b) {
+  if constexpr (KR) return b * prm.kb_rpb + prm.kb_off + (p - prm.key_lo);
+  else return kv_tensor_row(p, b, int32_t(prm.S), int32_t(prm.C), prm.B, prm.D, prm.kv_shard_major);
 }
 
 
@@ -121,7 +158,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int HD>
+template <int HD, bool KR>
 __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
     zsa_fwd_kernel(const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_k,
@@ -202,7 +239,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         unit_ring[slot] = idx;
         mbar_arrive(&bars.unit_full[slot]);
         if (idx < 0) break;
-        const UnitInfo u = load_unit(prm.units, idx);
+        const UnitInfo u = load_unit<HD, KR>(prm.units, idx, prm);
         for (int s = 0; s < NSLOT && ok; ++s) {
           if (u.kend[s] == 0) continue;
           if (q_fills[s] > 0) ok = mbar_wait(&bars.q_empty[s], (q_fills[s] - 1) & 1, wctx);
@@ -225,15 +262,14 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             if (use > 0) ok = mbar_wait(&bars.k_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.k_full[st], Cfg::KV_BYTES);
-            if (prm.kv_box == BK) {       // the tile's rows are contiguous: one box per d block
-              const int32_t krow = kv_tensor_row(n * BK, u.b, int32_t(prm.S), int32_t(prm.C),
-                                                 prm.B, prm.D, prm.kv_shard_major);
+            if (KR || prm.kv_box == BK) { // the tile's rows are contiguous: one box per d block
+              const int32_t krow = kv_row<KR>(prm, (u.n0 + n) * BK, u.b);
               for (int kb = 0; kb < KB; ++kb)
                 tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128, &map_k,
                             &bars.k_full[st], kb * 64, u.g, krow);
             } else {                      // 64-key boxes, one zigzag chunk each
               for (int hb = 0; hb < BK / 64; ++hb) {
-                const int32_t krow = kv_tensor_row(n * BK + hb * 64, u.b, int32_t(prm.S),
+                const int32_t krow = kv_tensor_row((u.n0 + n) * BK + hb * 64, u.b, int32_t(prm.S),
                                                    int32_t(prm.C), prm.B, prm.D, prm.kv_shard_major);
                 for (int kb = 0; kb < KB; ++kb)
                   tma_load_3d(smem + Cfg::SMEM_K + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
@@ -249,15 +285,14 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
             if (use > 0) ok = mbar_wait(&bars.v_empty[st], (use - 1) & 1, wctx);
             if (!ok) break;
             mbar_expect_tx(&bars.v_full[st], Cfg::KV_BYTES);
-            if (prm.kv_box == BK) {
-              const int32_t vrow = kv_tensor_row((n - 1) * BK, u.b, int32_t(prm.S), int32_t(prm.C),
-                                                 prm.B, prm.D, prm.kv_shard_major);
+            if (KR || prm.kv_box == BK) {
+              const int32_t vrow = kv_row<KR>(prm, (u.n0 + n - 1) * BK, u.b);
               for (int kb = 0; kb < KB; ++kb)
                 tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128, &map_v,
                             &bars.v_full[st], kb * 64, u.g, vrow);
             } else {
               for (int hb = 0; hb < BK / 64; ++hb) {
-                const int32_t vrow = kv_tensor_row((n - 1) * BK + hb * 64, u.b, int32_t(prm.S),
+                const int32_t vrow = kv_tensor_row((u.n0 + n - 1) * BK + hb * 64, u.b, int32_t(prm.S),
                                                    int32_t(prm.C), prm.B, prm.D, prm.kv_shard_major);
                 for (int kb = 0; kb < KB; ++kb)
                   tma_load_3d(smem + Cfg::SMEM_V + st * Cfg::KV_BYTES + kb * BK * 128 + hb * 64 * 128,
@@ -303,7 +338,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         const int idx = *reinterpret_cast<volatile int*>(&unit_ring[slot]);
         mbar_arrive(&bars.unit_empty[slot]);
         if (idx < 0) break;
-        const UnitInfo u = load_unit(prm.units, idx);
+        const UnitInfo u = load_unit<HD, KR>(prm.units, idx, prm);
         const int k0 = u.kend[0], k1 = NSLOT == 2 ? u.kend[1] : 0;
         // (n, s) walk over present pairs; first / last: s opens / closes key tile n
         int n = 0, sl = k0 > 0 ? 0 : 1;
@@ -405,8 +440,21 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.unit_empty[slot]);
       if (idx < 0) break;
-      const UnitInfo u = load_unit(prm.units, idx);
-      if (u.kend[s] == 0) continue;
+      const UnitInfo u = load_unit<HD, KR>(prm.units, idx, prm);
+      if (u.kend[s] == 0) {
+        if constexpr (KR) {
+          // a q tile that sees no key of the block: O = 0, lse = -inf, no MMA involved
+          if ((u.live >> s) & 1u) {
+            const int64_t j = int64_t(u.tile[s]) * 128 + row;
+            const int64_t rb = int64_t(u.r - prm.shard_begin) * prm.B + u.b;
+            uint4* dst = reinterpret_cast<uint4*>(prm.o + ((rb * twoC + j) * prm.Hq + u.head[s]) * HD);
+#pragma unroll 4
+            for (int v4 = 0; v4 < HD / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+            prm.lse[(rb * prm.Hq + u.head[s]) * twoC + j] = -INFINITY;
+          }
+        }
+        continue;
+      }
       const int64_t j = int64_t(u.tile[s]) * 128 + row;             // row within the shard
       const int64_t pos = j < prm.C ? int64_t(u.r) * prm.C + j
                                     : int64_t(2 * prm.D - 1 - u.r) * prm.C + (j - prm.C);
@@ -427,14 +475,30 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         // Causal mask on the tiles that cross this warp's diagonal only: keys past
         // `lim` (relative to the tile) are invisible to this row.  Off-diagonal tiles
         // (all but about one in kend) skip the mask entirely.
-        const int64_t rel = pos - int64_t(n) * BK;
-        const int lim = rel >= BK ? BK : int(rel);              // >= 0: key 0 is always visible
-        if (prm.causal && __any_sync(0xffffffffu, lim < BK - 1)) {
+        if constexpr (!KR) {
+          const int64_t rel = pos - int64_t(n) * BK;
+          const int lim = rel >= BK ? BK : int(rel);            // >= 0: key 0 is always visible
+          if (prm.causal && __any_sync(0xffffffffu, lim < BK - 1)) {
 #pragma unroll
-          for (int c = 0; c < BK / 32; ++c)
+            for (int c = 0; c < BK / 32; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e > lim) sr[c][e] = 0xFF800000u;    // -inf
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e > lim) sr[c][e] = 0xFF800000u;  // -inf
+          }
+        } else {
+          // visible: keys e of the tile with lo <= e <= hi (the block's bounds, and the
+          // causal limit); a row may see none of them (lo > hi)
+          const int32_t k0 = (u.n0 + n) * BK;
+          int hi = prm.key_hi - k0 - 1;
+          if (prm.causal && pos - k0 < hi) hi = int(pos - k0);
+          const int lo = prm.key_lo - k0;
+          if (__any_sync(0xffffffffu, lo > 0 || hi < BK - 1)) {
+#pragma unroll
+            for (int c = 0; c < BK / 32; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e > hi || c * 32 + e < lo) sr[c][e] = 0xFF800000u;
+          }
         }
         // row max of the raw scores (three-input max, four independent chains)
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -461,7 +525,10 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
         // consumes (normalises O, keeping it a convex combination of V rows: exact when
         // one key dominates a row).
         const uint64_t scale2 = f2_pack(prm.scale_log2, prm.scale_log2);
-        const uint64_t negm2 = f2_pack(-m_run, -m_run);
+        // a row with no visible key so far keeps m = -inf; it subtracts 0 instead (its
+        // P is exactly 0 either way)
+        const float m_sub = (KR && m_run == -INFINITY) ? 0.f : m_run;
+        const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
         uint64_t lsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
         uint64_t rsum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
         uint32_t pk[BK / 32][16];
@@ -518,7 +585,8 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
       o_ph ^= 1;
       if (!ok) break;
       tc_fence_after();
-      const float inv_l = 1.0f / r_run;
+      // a row that saw no key of the block (key-block launches only): O = 0, lse = -inf
+      const float inv_l = (KR && r_run == 0.f) ? 0.f : 1.0f / r_run;
       const int64_t rb = int64_t(u.r - prm.shard_begin) * prm.B + u.b;   // local (shard, b)
       const int64_t grow = rb * twoC + j;                                 // shard-major row
       __nv_bfloat16* orow_g = prm.o + (grow * prm.Hq + u.head[s]) * HD;
@@ -538,7 +606,7 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
           dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
       }
       prm.lse[(rb * prm.Hq + u.head[s]) * twoC + j] =
-          (m_run + log2f(l_run)) * 0.69314718055994530942f;
+          (KR && l_run == 0.f) ? -INFINITY : (m_run + log2f(l_run)) * 0.69314718055994530942f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.o_empty[s]);
@@ -551,11 +619,12 @@ __global__ void __launch_bounds__(FwdCfg<HD>::NTHREADS, 1)
   if (warp == Cfg::WARP_MMA) tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
-template <int HD>
+template <int HD, bool KR>
 int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   using Cfg = FwdCfg<HD>;
   const int64_t rows = int64_t(a.shard_count) * a.B * (a.S / a.D);  // local shard-major rows
-  const int32_t kv_box = (a.S / (2 * int64_t(a.D))) % Cfg::BK == 0 ? Cfg::BK : 64;
+  const int32_t kv_box = KR || (a.S / (2 * int64_t(a.D))) % Cfg::BK == 0 ? Cfg::BK : 64;
+  const uint64_t kv_rows = KR ? uint64_t(a.kv_rows) : uint64_t(a.B * a.S);
   CUtensorMap mq, mk, mv;
   {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hq), uint64_t(rows)};
@@ -564,7 +633,7 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
     if (!make_map_bf16_sw128(&mq, a.q, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
   {
-    const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), uint64_t(a.B * a.S)};
+    const uint64_t dims[3] = {uint64_t(HD), uint64_t(a.Hkv), kv_rows};
     const uint64_t strides[2] = {uint64_t(HD) * 2, uint64_t(a.Hkv) * HD * 2};
     // a box never straddles a zigzag chunk: the K/V rows it covers are contiguous in
     // both layouts
@@ -580,17 +649,24 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   p.S = a.S;
   p.C = a.S / (2 * int64_t(a.D));
   p.B = a.B; p.Hq = a.Hq; p.Hkv = a.Hkv; p.D = a.D; p.causal = a.causal;
-  p.kv_shard_major = a.kv_layout;
   p.shard_begin = a.shard_begin;
-  p.kv_box = kv_box;
+  if (KR) {
+    p.kb_rpb = a.kv_rows_per_batch;
+    p.kb_off = a.kv_row_offset;
+  } else {
+    p.kv_shard_major = a.kv_layout;
+    p.kv_box = kv_box;
+  }
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
   p.status = a.status;
   p.counter = a.status + 32;
   p.wait_limit_ns = a.wait_limit_ns;
   p.inject_stall = a.inject_stall;
+  p.key_lo = a.key_lo;
+  p.key_hi = a.key_hi;
   const int smem = Cfg::SMEM_BYTES + 1024;
   {
-    const int e = ensure_smem_attr(reinterpret_cast<const void*>(zsa_fwd_kernel<HD>), smem);
+    const int e = ensure_smem_attr(reinterpret_cast<const void*>(zsa_fwd_kernel<HD, KR>), smem);
     if (e != int(cudaSuccess)) return e;
   }
   int dev = 0, sms = 148;
@@ -600,7 +676,7 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
   if (grid <= 0) return int(cudaSuccess);
   const TraceEvents tr = trace_events(0);
   if (tr.begin) cudaEventRecord(tr.begin, stream);
-  zsa_fwd_kernel<HD><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, p);
+  zsa_fwd_kernel<HD, KR><<<grid, Cfg::NTHREADS, smem, stream>>>(mq, mk, mv, p);
   const cudaError_t e = cudaGetLastError();
   if (tr.end) cudaEventRecord(tr.end, stream);
   return int(e);
@@ -610,9 +686,9 @@ int launch_fwd_hd(const FwdArgs& a, cudaStream_t stream) {
 
 int launch_fwd(const FwdArgs& a, cudaStream_t stream) {
   switch (a.d) {
-    case 64: return launch_fwd_hd<64>(a, stream);
-    case 128: return launch_fwd_hd<128>(a, stream);
-    case 256: return launch_fwd_hd<256>(a, stream);
+    case 64: return a.key_block ? launch_fwd_hd<64, true>(a, stream) : launch_fwd_hd<64, false>(a, stream);
+    case 128: return a.key_block ? launch_fwd_hd<128, true>(a, stream) : launch_fwd_hd<128, false>(a, stream);
+    case 256: return a.key_block ? launch_fwd_hd<256, true>(a, stream) : launch_fwd_hd<256, false>(a, stream);
     default: return int(cudaErrorInvalidValue);
   }
 }

@@ -24,6 +24,12 @@ struct FwdArgs {
   int* status;
   uint64_t wait_limit_ns;
   int inject_stall;        // test hook: the MMA threads first wait on a barrier nobody arrives at
+  // key-block launch (key_block != 0): only keys at positions [key_lo, key_hi) count, and
+  // K/V are a [kv_rows][Hkv][d] tensor holding the key at position p of batch b in row
+  // b * kv_rows_per_batch + kv_row_offset + p - key_lo (kv_layout is not used)
+  int32_t key_block = 0;
+  int32_t key_lo = 0, key_hi = 0;
+  int32_t kv_rows_per_batch = 0, kv_row_offset = 0, kv_rows = 0;
 };
 
 struct BwdArgs {
@@ -51,6 +57,16 @@ struct BwdArgs {
 // Partial results to merge (ring attention): n parts of the Q layout (bf16 O) and the
 // lse layout (fp32), rows = local Q-layout rows of the problem.
 constexpr int kMergeMaxParts = 32;
+// K5: natural [B][S][H][d] <-> shard-major [shards][B][2C][H][d] copy (bf16 rows).
+struct PermuteArgs {
+  const void* src;
+  void* dst;
+  int64_t chunk_words;     // 16-byte words in one chunk of one batch: C * H * d * 2 / 16
+  int32_t B, D;
+  int32_t shard_begin, shard_count;
+  int32_t to_shard_major;  // 1: src natural, dst shard-major; 0: the reverse
+};
+
 struct MergeArgs {
   const void* o[kMergeMaxParts];
   const float* lse[kMergeMaxParts];
@@ -91,7 +107,7 @@ struct TraceEvents {
   cudaEvent_t begin, end;
 };
 TraceEvents trace_events(int which);  // 0 fwd, 1 bwd pre, 2 bwd main, 3 dQ convert, 4 merge,
-                                      // 5 projection GEMM
+                                      // 5 projection GEMM, 6 permute
 
 // Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once
 // per (kernel, device): cudaFuncSetAttribute applies to the device current at the time
@@ -107,6 +123,7 @@ int inject_stall();
 int launch_fwd(const FwdArgs& a, cudaStream_t stream);
 int launch_bwd(const BwdArgs& a, cudaStream_t stream);
 int launch_merge(const MergeArgs& a, cudaStream_t stream);
+int launch_permute(const PermuteArgs& a, cudaStream_t stream);
 int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream);
 
 }  // namespace zsa

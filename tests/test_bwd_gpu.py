@@ -25,12 +25,12 @@ CASES = [  # (B, S, Hq, Hkv, d, D, causal, seed)
     (1, 1536, 4, 1, 128, 3, True, 6),      # GQA 4, D = 3
     (1, 1024, 4, 4, 128, 1, True, 7),      # D = 1
     (1, 2048, 4, 2, 64, 8, True, 8),       # D = 8
-    (1, 1024, 6, 1, 256, 2, True, 9),      # d = 256 (two d-chunk units per key tile), GQA 6
-    (1, 512, 4, 2, 256, 2, True, 10),      # d = 256, 32-row q slots, C = 128
+    (1, 1024, 6, 1, 256, 2, True, 9),      # d = 256 (two-CTA cluster per key tile), GQA 6
+    (1, 512, 4, 2, 256, 2, True, 10),      # d = 256, 64-row q slots, C = 128
     (2, 512, 2, 2, 256, 1, False, 11),     # d = 256, non-causal, D = 1, B = 2
     # more units than CTAs, so every CTA carries state from one key tile to the next
     (1, 4096, 16, 8, 64, 4, True, 12),     # 256 units (d = 64)
-    (1, 4096, 6, 1, 256, 4, True, 13),     # 64 key tiles x 2 d chunks, 4096-long slot walks
+    (1, 4096, 6, 1, 256, 4, True, 13),     # 32 key tiles over the clusters, long slot walks
 ]
 
 

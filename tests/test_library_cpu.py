@@ -104,3 +104,50 @@ def test_argument_errors(L):
                          ctypes.cast(sched, ctypes.c_void_p), 1, ctypes.byref(n))
     assert rc == zsa.ZSA_ERR_WORKSPACE and n.value > 1
     assert (t.block_q, t.block_k, t.slots) == (128, 128, 2)
+
+
+def test_permute_argument_errors(L):
+    good = zsa.make_problem(2, 1024, 4, 2, 128, 2)
+    P = ctypes.byref(good)
+    n = 2 * 1024 * 4 * 128 * 2                      # bytes of a [B][S][4][d] bf16 tensor
+    assert L.zsa_permute(P, 4, 1, 16, 16, None) == zsa.ZSA_ERR_INVALID          # overlap
+    assert L.zsa_permute(P, 4, 1, 16, 16 + n - 16, None) == zsa.ZSA_ERR_INVALID
+    # a shard range: the shard-major side is that range's rows only
+    one = zsa.make_problem(2, 1024, 4, 2, 128, 2, shard_begin=1, shard_count=1)
+    P1 = ctypes.byref(one)
+    assert L.zsa_permute(P1, 4, 1, 16 + n // 2 - 16, 16, None) == zsa.ZSA_ERR_INVALID
+    assert L.zsa_permute(P1, 4, 0, 16, 16 + n // 2 - 16, None) == zsa.ZSA_ERR_INVALID
+    # adjacent, not overlapping: passes the argument checks (then fails for want of a GPU)
+    assert L.zsa_permute(P1, 4, 1, 16 + n // 2, 16, None) not in (zsa.ZSA_OK, zsa.ZSA_ERR_INVALID)
+    assert L.zsa_permute(P1, 4, 0, 16, 16 + n // 2, None) not in (zsa.ZSA_OK, zsa.ZSA_ERR_INVALID)
+    assert L.zsa_permute(P, 4, 1, 16, 24 + n, None) == zsa.ZSA_ERR_INVALID       # misaligned
+    assert L.zsa_permute(P, 0, 1, 16, 16 + n, None) == zsa.ZSA_ERR_INVALID       # heads
+    assert L.zsa_permute(P, 4, 2, 16, 16 + n, None) == zsa.ZSA_ERR_INVALID       # direction
+    assert L.zsa_permute(P, 4, 1, None, 16 + n, None) == zsa.ZSA_ERR_INVALID
+    assert L.zsa_permute(None, 4, 1, 16, 16 + n, None) == zsa.ZSA_ERR_INVALID
+    bad = zsa.make_problem(1, 1000, 4, 2, 128, 2)
+    assert L.zsa_permute(ctypes.byref(bad), 4, 1, 16, 16 + n, None) == zsa.ZSA_ERR_SHAPE
+    big = zsa.make_problem(40000, 1024, 4, 2, 128, 2)
+    assert L.zsa_permute(ctypes.byref(big), 1, 1, 16, 1 << 40, None) == zsa.ZSA_ERR_SHAPE
+
+
+def test_key_block_argument_errors(L):
+    # B = 2, S = 1024: a compact block of keys [100, 612) needs 2 * 512 rows
+    good = zsa.make_problem(2, 1024, 4, 2, 128, 2)
+
+    def rc(lo, hi, rpb, off, rows, ws_bytes=64):
+        kb = zsa.zsa_key_block(lo, hi, rpb, off, rows)
+        return L.zsa_attn_fwd_block(ctypes.byref(good), ctypes.byref(kb), *((16,) * 5), 256,
+                                    ws_bytes, None)
+
+    assert rc(100, 612, 512, 0, 1024) == zsa.ZSA_ERR_WORKSPACE      # valid: reaches the size check
+    assert rc(0, 0, 0, 0, 1) == zsa.ZSA_ERR_WORKSPACE               # an empty block is valid
+    assert rc(100, 612, 512, 0, 1023) == zsa.ZSA_ERR_INVALID        # last row outside the tensor
+    assert rc(100, 612, 511, 0, 4096) == zsa.ZSA_ERR_INVALID        # batches overlap
+    assert rc(612, 100, 512, 0, 1024) == zsa.ZSA_ERR_INVALID        # hi < lo
+    assert rc(-1, 100, 512, 0, 1024) == zsa.ZSA_ERR_INVALID
+    assert rc(0, 1025, 1025, 0, 4096) == zsa.ZSA_ERR_INVALID        # past S
+    assert rc(0, 100, 100, -1, 1024) == zsa.ZSA_ERR_INVALID
+    assert rc(0, 100, 100, 0, 1 << 31) == zsa.ZSA_ERR_INVALID       # int32 TMA coordinates
+    assert L.zsa_attn_fwd_block(ctypes.byref(good), None, *((16,) * 5), 256, 1 << 30,
+                                None) == zsa.ZSA_ERR_INVALID
