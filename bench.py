@@ -52,11 +52,7 @@ DEFAULT_CONFIG = "long"
 # the current kernel at the configuration's full size (dram__bytes_read.sum +
 # dram__bytes_write.sum, a one-pass capture; profiles/dram_traffic_bwd_main.md);
 # configurations without a capture report null.
-MEASURED_TRAFFIC = {
-    ("long", "zsa_bwd_wide_kernel"): 18.71e9 + 10.49e9,
-    ("8b_gqa", "zsa_bwd_wide_kernel"): 1.954867e9 + 1.042157e9,
-    ("wide_gqa", "zsa_bwd_pair_kernel"): 38.77e9 + 22.84e9,
-}
+MEASURED_TRAFFIC = {}
 # Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
 CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
 
@@ -363,7 +359,8 @@ def run_zsa(args, c, name):
     traffic = MEASURED_TRAFFIC.get((name, dom))
     # the two HBM-bound kernels: algorithmic bytes per launch over their event time
     pairs = B * S * Hq // world
-    pre_bytes = pairs * (2 * d * 2 + 4 + 4 * d)    # read O, dO; write Delta, zero dQacc
+    # read O, dO, lse; write -Delta, -lse log2(e), the zeroed dQacc
+    pre_bytes = pairs * (2 * d * 2 + 4 + 4 + 4 + 4 * d)
     dqc_bytes = pairs * d * (4 + 2)                # read fp32 dQacc; write bf16 dQ
     hbm_kernels = {
         "bwd_pre": {"bytes": pre_bytes, "gbs": pre_bytes / (kms[1] * 1e-3) / 1e9,

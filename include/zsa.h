@@ -146,8 +146,9 @@ ZSA_API int zsa_partition(const zsa_problem* problem, zsa_tiling* tiling, int32_
  * No passage defines it: the caller owns all device memory, so the library states how
  * much scratch each pass needs.
  * The workspace must be device memory, 256-byte aligned, not shared between calls in
- * flight.  fwd: status word + the unit table.  bwd: status word + Delta (fp32
- * [D][B][Hq][2C]) + a dQ accumulator (fp32, head-major [Hq][D*B*2C][d]). */
+ * flight.  fwd: status word + the unit table.  bwd: status word + -Delta and
+ * -lse*log2(e) (fp32 [D][B][Hq][2C] each) + a dQ accumulator (fp32, head-major
+ * [Hq][D*B*2C][d]). */
 ZSA_API int zsa_workspace_bytes(const zsa_problem* problem, int pass, size_t* bytes_out);
 
 /* Forward: o (bf16, Q layout) and lse (fp32 [D][B][Hq][2C]).  q, k, v, o, lse and the

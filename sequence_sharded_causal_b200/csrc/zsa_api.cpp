@@ -135,9 +135,9 @@ size_t fwd_workspace(const zsa_problem* p) {
 }
 
 size_t bwd_workspace(const zsa_problem* p) {
-  const size_t stats = size_t(local_rows(p)) * p->Hq * sizeof(float);       // Delta
+  const size_t stats = size_t(local_rows(p)) * p->Hq * sizeof(float);  // -Delta, -lse log2 e
   const size_t dqacc = size_t(local_rows(p)) * p->Hq * p->d * sizeof(float);
-  return kStatusBytes + align256(stats) + align256(dqacc);
+  return kStatusBytes + 2 * align256(stats) + align256(dqacc);
 }
 
 }  // namespace
@@ -366,7 +366,8 @@ int zsa_attn_bwd(const zsa_problem* problem, const void* q, const void* k, const
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.delta = reinterpret_cast<float*>(ws + kStatusBytes);
-  a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes + align256(stats));
+  a.nlse2 = reinterpret_cast<float*>(ws + kStatusBytes + align256(stats));
+  a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes + 2 * align256(stats));
   a.S = problem->S; a.B = int32_t(problem->B); a.Hq = problem->Hq; a.Hkv = problem->Hkv;
   a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
   a.scale = problem->softmax_scale;

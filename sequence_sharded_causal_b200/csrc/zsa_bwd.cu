@@ -7,7 +7,7 @@
 //   per key tile (b, kv head g, n), over every (shard, q tile, q head of g) that sees it:
 //     S^T = K Q^T,  P^T = exp(scale S^T - lse),  dP^T = V dO^T,
 //     dS^T = P^T * (dP^T - Delta),
-//     dV += P^T dO,  dK += dS^T Q,  dQ^T (+)= K^T dS^T                 (K3, tensor-bound)
+//     dV += P^T dO,  dK += dS^T Q,  dQ (+)= dS K                       (K3, tensor-bound)
 //   dQ = bf16(scale * dQacc)                                          (K4, HBM-bound)
 // dK and dV are summed over every shard and the G q heads of the group inside one CTA
 // (the single-GPU stand-in for the reduce-scatter back to the owning shards); dQ is
@@ -16,7 +16,7 @@
 // K3 has two builds, chosen by head dim.  Both claim 128-key-tile units (b, kv head, key
 // tile) from a global counter in that order, keep the unit's K and V tiles in shared
 // memory, stream the q slots that see the tile through a TMA ring (Q, dO, lse, Delta),
-// send dQ^T through shared memory into TMA bulk reduce-adds, and bound every wait.
+// send dQ through shared memory into TMA bulk reduce-adds, and bound every wait.
 //
 //  zsa_bwd_wide_kernel (d <= 128, this file): one CTA per key tile;
 //   * 128-row q slots, so all five MMAs of a slot are N = 128; a 128-row slot may
@@ -24,15 +24,16 @@
 //     rows, each over contiguous positions;
 //   * TMEM: dV | dK (fp32, lanes = keys) | ST | XT.  ST receives S^T, then the bf16 P^T
 //     and dS^T (TMEM A operands of dV and dK); XT receives dP^T and, once the compute
-//     warps have read it, dQ^T = K^T dS^T (A = the resident K tile read MN-major, B =
-//     dS^T in shared memory);
-//   * two MMA-issuing threads: one issues S^T and dP^T, the other dV, dK and dQ^T;
-//   * 4 dQ warps stage dQ^T in the slot's own Q / dO stage and reduce it into the fp32
-//     accumulator.
+//     warps have read it, dQ = dS K (A = dS^T in shared memory read M-major, B = the
+//     resident K tile read N-major), so a TMEM lane is a q row;
+//   * two MMA-issuing threads: one issues S^T and dP^T, the other dV, dK and dQ;
+//   * 4 dQ warps stage dQ, a q row per thread, in the slot's own Q / dO stage and
+//     reduce it into the fp32 accumulator.
 //
 //  zsa_bwd_pair_kernel (d = 256, zsa_bwd_pair.cu): a cluster of two CTAs per key tile,
 //  one holding K and dK, the other V and dV, exchanging P^T and dS^T through
-//  distributed shared memory (dK + dV of the tile alone would fill one SM's TMEM).
+//  distributed shared memory (dK + dV of the tile alone would fill one SM's TMEM); it
+//  computes dQ transposed, dQ^T = K^T dS^T, in two 128-row d halves.
 #include <cuda_bf16.h>
 
 #include "zsa_bwd_common.cuh"
@@ -46,10 +47,16 @@ using namespace bwd;
 
 
 // ------------------------------------------------------------------ K2: Delta + zero dQacc
+// Per (row, head): -Delta = -rowsum(dO * O) and -lse * log2(e), the two per-row terms of
+// the main kernel's element formulas stored ready to add (P^T = 2^(scale log2(e) S^T +
+// (-lse log2 e)) is one FMA, dS^T = P^T (dP^T + (-Delta)) one add and one multiply), and
+// the zeroed dQ accumulator.
 template <int HD>
 __global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                           const __nv_bfloat16* __restrict__ dout,
-                                                          float* __restrict__ delta,
+                                                          const float* __restrict__ lse,
+                                                          float* __restrict__ ndelta,
+                                                          float* __restrict__ nlse2,
                                                           float* __restrict__ dq_acc,
                                                           int64_t n_pairs, int32_t Hq,
                                                           int64_t twoC) {
@@ -85,7 +92,9 @@ __global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* _
       const int64_t row = pair / Hq;           // (r*B + b)*2C + j
       const int32_t h = int32_t(pair % Hq);
       const int64_t rb = row / twoC, j = row % twoC;
-      delta[(rb * Hq + h) * twoC + j] = acc;
+      const int64_t sidx = (rb * Hq + h) * twoC + j;
+      ndelta[sidx] = -acc;
+      nlse2[sidx] = -lse[sidx] * kLog2e;
     }
   }
 }
@@ -121,7 +130,7 @@ __global__ void __launch_bounds__(256) zsa_dq_convert_kernel(const float* __rest
 // its rate on N = 64 shapes whose operands all come from shared memory).  TMEM holds
 // dV | dK | ST | XT: ST receives S^T and then the bf16 P^T and dS^T (half its columns
 // each, A operands of dV and dK); XT receives dP^T and, once the compute warps have
-// loaded it, dQ^T.  One slot is in flight; the next slot's S^T is issued as soon as
+// loaded it, dQ.  One slot is in flight; the next slot's S^T is issued as soon as
 // dK has consumed ST, its dP^T as soon as the dQ warps have read XT.
 template <int HD>
 struct BwdWideCfg {
@@ -143,7 +152,7 @@ struct BwdWideCfg {
   static constexpr int WARP_DQ = 8;
   static constexpr int WARP_LOAD = 12;
   static constexpr int WARP_MMA = 13;   // S^T, dP^T issuer (and TMEM owner)
-  static constexpr int WARP_MMA2 = 14;  // dV, dK, dQ^T issuer
+  static constexpr int WARP_MMA2 = 14;  // dV, dK, dQ issuer
   static constexpr int NTHREADS = 15 * 32;
   static constexpr uint32_t TM_DV = 0;
   static constexpr uint32_t TM_DK = HD;
@@ -193,8 +202,8 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     mbar_init(&bars.kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.q_full[s], 1);
-      // 8 compute warps (lse / Delta read) + 4 dQ warps (their reduce has read the
-      // dQ^T staged in this stage's Q / dO space, after every MMA of the slot)
+      // 8 compute warps (lse / Delta read) + 4 dQ warps (their reduces have read the
+      // dQ staged in this stage's Q / dO space, after every MMA of the slot)
       mbar_init(&bars.q_empty[s], 8 + 4);
     }
     mbar_init(&bars.s_full, 1);
@@ -280,8 +289,8 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
                         &bars.q_full[st], kb * 64, h, row0);
           }
           const int64_t stat = (rb * prm.Hq + h) * twoC + int64_t(w.i) * BQ;
-          bulk_load(smem + Cfg::SMEM_LSE + st * BQ * 4, prm.lse + stat, BQ * 4, &bars.q_full[st]);
-          bulk_load(smem + Cfg::SMEM_DELTA + st * BQ * 4, prm.delta + stat, BQ * 4, &bars.q_full[st]);
+          bulk_load(smem + Cfg::SMEM_LSE + st * BQ * 4, prm.nlse2 + stat, BQ * 4, &bars.q_full[st]);
+          bulk_load(smem + Cfg::SMEM_DELTA + st * BQ * 4, prm.ndelta + stat, BQ * 4, &bars.q_full[st]);
           ++q_fills[st];
           ++q_it;
         }
@@ -296,7 +305,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
   } else if (warp == Cfg::WARP_MMA || warp == Cfg::WARP_MMA2) {
     // ------------------------------------------------------------ MMA issuers
     // Thread A (WARP_MMA) issues each slot's S^T and dP^T, thread B (WARP_MMA2) its dV,
-    // dK and dQ^T.  Their TMEM hand-offs are barriers already (st_free: B's dK has
+    // dK and dQ.  Their TMEM hand-offs are barriers already (st_free: B's dK has
     // consumed ST; dq_empty: the dQ warps have read XT; ds_full: the compute warps have
     // read dP^T), so neither waits on the other's issue order, and one thread's barrier
     // latency no longer idles the tensor pipe.  tcgen05.commit tracks the issuing
@@ -307,15 +316,12 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
       const bool role_a = warp == Cfg::WARP_MMA;
       const uint32_t idesc_s = idesc_bf16(128, BQ, false, false);   // S^T, dP^T
       const uint32_t idesc_kv = idesc_bf16(128, HD, false, true);   // dV, dK (A from TMEM)
-      const uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);    // dQ^T
+      const uint32_t idesc_dq = idesc_bf16(BQ, HD, true, true);     // dQ = dS K
       const uint32_t sK = smem_u32(smem + Cfg::SMEM_K);
       const uint32_t sV = smem_u32(smem + Cfg::SMEM_V);
       const uint32_t sQ = smem_u32(smem + Cfg::SMEM_Q);
       const uint32_t sDO = smem_u32(smem + Cfg::SMEM_DO);
       const uint32_t sDS = smem_u32(smem + Cfg::SMEM_DS);
-      // dQ^T = K^T dS^T: A = K^T (M = d in 64-row blocks at the K tile's d-block stride;
-      // with d = 64 the second M block reads V and its rows are never used)
-      const uint32_t lbo_kt = HD >= 128 ? uint32_t(BKV * 128) : uint32_t(Cfg::SMEM_V - Cfg::SMEM_K);
       uint32_t kv_ph = 0, q_it = 0, p_ph = 0, ds_ph = 0;
       uint32_t q_full_uses[2] = {0, 0};
       uint32_t st_waits = 0, xt_waits = 0, acc_commits = 0;
@@ -355,7 +361,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
                        sdesc_sw128(sQ + st * Cfg::QT_BYTES + kb * BQ * 128 + ks * 32, 16, 1024),
                        idesc_s, (kb | ks) != 0);
             mma_commit(&bars.s_full);
-            // dP^T into XT once the dQ warps have read the previous dQ^T out of it
+            // dP^T into XT once the dQ warps have read the previous dQ out of it
             if (q_it > 0) ok = mbar_wait(&bars.dq_empty, xt_waits++ & 1, wctx);
             if (!ok) break;
             tc_fence_after();
@@ -378,7 +384,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
               mma_ts(tmem + Cfg::TM_DV, tmem + Cfg::TM_ST + p_col(ks),
                      sdesc_sw128(sDO + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
                      !j0 || (ks > 0));
-            // dK += dS^T Q, then dQ^T = K^T dS^T into XT (dP^T there was loaded already)
+            // dK += dS^T Q, then dQ = dS K into XT (dP^T there was loaded already)
             ok = mbar_wait(&bars.ds_full, ds_ph, wctx);
             ds_ph ^= 1;
             if (!ok) break;
@@ -389,13 +395,15 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
                      sdesc_sw128(sQ + st * Cfg::QT_BYTES + ks * 2048, BQ * 128, 1024), idesc_kv,
                      !j0 || (ks > 0));
             mma_commit(&bars.st_free);
+            // A = dS: the dS^T tile read M-major (two 64-wide q blocks 16 KB apart);
+            // B = K: the resident K tile read N-major (64-wide d blocks 16 KB apart)
 #pragma unroll
             for (int ks = 0; ks < BKV / 16; ++ks)
-              mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sK + ks * 2048, lbo_kt, 1024),
-                     sdesc_sw128(sDS + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
+              mma_ss(tmem + Cfg::TM_XT, sdesc_sw128(sDS + ks * 2048, BKV * 128, 1024),
+                     sdesc_sw128(sK + ks * 2048, BKV * 128, 1024), idesc_dq, ks > 0);
             mma_commit(&bars.dq_full);
             mma_commit(&bars.dsm_free);
-            // the stage's Q / dO are released by the dQ warps, which stage dQ^T there
+            // the stage's Q / dO are released by the dQ warps, which stage dQ there
           }
           ++q_it;
         }
@@ -412,16 +420,21 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
     __syncwarp();
   } else if (warp >= Cfg::WARP_DQ) {
     // ------------------------------------------------------------ dQ warps
-    // dQ^T of a slot (TMEM lane = d index, column = q row) goes from TMEM to shared
-    // memory and from there into the fp32 accumulator by one TMA bulk reduce-add per
-    // warp: warp qw stages d rows 32qw .. 32qw+31 as a [128 q][32 d] fp32 box (128-byte
-    // rows, 128-byte swizzle).  The staging space is the slot's own Q and dO stage
-    // (HD * 512 bytes, exactly the size of dQ^T): once dQ^T is ready every MMA that reads
-    // that stage has completed, and the producer refills it only after the reduces have
-    // read it out (q_empty).  No per-element atomics leave the SM.
+    // dQ = dS K of a slot lies in XT with TMEM lane = q row and column = d, so dQ warp
+    // qw holds q rows 32qw .. 32qw+31 and each thread one row: it moves its row in 16-byte
+    // pieces into [32 q][32 d] fp32 boxes (128-byte rows, 128-byte swizzle: conflict-free
+    // for 8 threads a wavefront) and one TMA bulk reduce-add per box adds them into the
+    // head-major fp32 accumulator.  The boxes live in the slot's own Q and dO stage (HD *
+    // 512 bytes, exactly the size of dQ): once dQ exists every MMA that reads that stage
+    // has completed, and the producer refills it only after the reduces have read it out
+    // (q_empty).  XT is read in pairs of 32-column chunks and released after the last
+    // pair's load, before that pair is staged.  No per-element atomics leave the SM.
     const int qw = warp - Cfg::WARP_DQ;
     const uint32_t tXT = tmem + Cfg::TM_XT + (uint32_t(qw * 32) << 16);
-    const bool has_box = qw * 32 < HD;
+    constexpr int NCH = HD / 32;                   // 32-column chunks of a row of dQ
+    uint32_t sw_off[8];                            // this thread's row, 16-byte piece j
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sw_off[j] = sw128_offset(uint32_t(lane), uint32_t(j));
     uint32_t dq_ph = 0, q_it = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -440,38 +453,39 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const int st = int(q_it & 1);
-        uint8_t* box = qw < KB ? smem + Cfg::SMEM_Q + st * Cfg::QT_BYTES + qw * (BQ * 128)
-                               : smem + Cfg::SMEM_DO + st * Cfg::QT_BYTES + (qw - KB) * (BQ * 128);
+        const int32_t h = u.g * prm.G + w.e;
+        const int32_t row0 = int32_t((int64_t(w.r - prm.shard_begin) * prm.B + u.b) * twoC +
+                                     int64_t(w.i) * BQ + qw * 32);
 #pragma unroll 1
-        for (int t = 0; t < BQ / 32; ++t) {
-          uint32_t v[32];
-          tmem_ld32(tXT + t * 32, v);
+        for (int c0 = 0; c0 < NCH; c0 += 2) {
+          uint32_t v[2][32];
+          tmem_ld32(tXT + c0 * 32, v[0]);
+          tmem_ld32(tXT + c0 * 32 + 32, v[1]);
           tmem_ld_wait();
-          if (t + 1 == BQ / 32) {          // all of dQ^T read: XT may be overwritten
+          if (c0 + 2 == NCH) {             // all of dQ read: XT may be overwritten
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.dq_empty);
           }
-          if (has_box) {
-            const uint32_t within = uint32_t(lane & 3) * 4;
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              *reinterpret_cast<uint32_t*>(box + sw128_offset(uint32_t(t * 32 + c), uint32_t(lane >> 2)) +
-                                           within) = v[c];
+          for (int cc = 0; cc < 2; ++cc) {
+            const int bi = qw * NCH + c0 + cc;   // box index within the stage's 16*HD rows
+            uint8_t* box = bi * 4096 < Cfg::QT_BYTES
+                               ? smem + Cfg::SMEM_Q + st * Cfg::QT_BYTES + bi * 4096
+                               : smem + Cfg::SMEM_DO + st * Cfg::QT_BYTES + (bi * 4096 - Cfg::QT_BYTES);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(box + sw_off[j]) =
+                  make_uint4(v[cc][4 * j], v[cc][4 * j + 1], v[cc][4 * j + 2], v[cc][4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_3d(&map_dq, box, (c0 + cc) * 32, row0, h);
+              bulk_commit_group();
+            }
           }
         }
-        if (has_box) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            const int32_t h = u.g * prm.G + w.e;
-            const int32_t row0 =
-                int32_t((int64_t(w.r - prm.shard_begin) * prm.B + u.b) * twoC + int64_t(w.i) * BQ);
-            tma_reduce_add_3d(&map_dq, box, qw * 32, row0, h);
-            bulk_commit_group();
-            bulk_wait_group_read0();
-          }
-        }
+        if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.q_empty[st]);
         ++q_it;
@@ -513,11 +527,16 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         ok = warp_wait_b(&bars.q_full[st], q_full_uses[st] & 1, wctx);
         ++q_full_uses[st];
         if (!ok) break;
-        const float* lse_c = reinterpret_cast<const float*>(smem + Cfg::SMEM_LSE) + st * BQ + 64 * hgrp;
-        const float* dlt_c = reinterpret_cast<const float*>(smem + Cfg::SMEM_DELTA) + st * BQ + 64 * hgrp;
+        // this group's 64 columns of -lse log2(e) and -Delta (K2), as float4s
+        const float4* nl4 = reinterpret_cast<const float4*>(smem + Cfg::SMEM_LSE) + (st * BQ + 64 * hgrp) / 4;
+        const float4* nd4 = reinterpret_cast<const float4*>(smem + Cfg::SMEM_DELTA) + (st * BQ + 64 * hgrp) / 4;
         const int64_t p0 = zz_pos(prm.C, prm.D, w.r, int64_t(w.i) * BQ + 64 * hgrp);
         const int nvis_lo = prm.causal ? int(key - p0) : 0;   // columns c < nvis_lo are masked
-        // ---- P^T = exp(scale S^T - lse) -> bf16 over the first half of this group's columns
+        // only slots whose columns cross this warp's keys need the mask (warp-uniform)
+        const bool masked = __any_sync(0xffffffffu, nvis_lo > 0);
+        const uint64_t scale2 = f2_pack(prm.scale_log2, prm.scale_log2);
+        // ---- P^T = 2^(scale log2(e) S^T - lse log2(e)) -> bf16 over the first half of
+        //      this group's columns
         ok = warp_wait_b(&bars.s_full, s_ph, wctx);
         s_ph ^= 1;
         if (!ok) break;
@@ -529,12 +548,23 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
           tmem_ld32(tS + cc * 32, sv);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = cc * 32 + 2 * e;
-            const float x0 = fmaf(__uint_as_float(sv[2 * e]), prm.scale_log2, -lse_c[c0] * kLog2e);
-            const float x1 = fmaf(__uint_as_float(sv[2 * e + 1]), prm.scale_log2, -lse_c[c0 + 1] * kLog2e);
-            pk[cc][e] = pack_bf16x2(c0 < nvis_lo ? 0.f : ex2_approx(x0),
-                                    c0 + 1 < nvis_lo ? 0.f : ex2_approx(x1));
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 nl = nl4[cc * 8 + q4];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int e = 2 * q4 + hh;
+              const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                                         scale2, hh == 0 ? f2_pack(nl.x, nl.y) : f2_pack(nl.z, nl.w));
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+              if (masked) {
+                const int c0 = cc * 32 + 2 * e;
+                e0 = c0 < nvis_lo ? 0.f : e0;
+                e1 = c0 + 1 < nvis_lo ? 0.f : e1;
+              }
+              pk[cc][e] = pack_bf16x2(e0, e1);
+            }
           }
           tmem_st16(tS + cc * 16, pk[cc]);     // S^T columns already loaded
         }
@@ -543,7 +573,7 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.p_full);
         // ---- dS^T = P^T (dP^T - Delta) -> bf16 into the second half of the columns and
-        //      into shared memory (B operand of dQ^T)
+        //      into shared memory (A operand of dQ)
         ok = warp_wait_b(&bars.dp_full, dp_ph, wctx);
         dp_ph ^= 1;
         if (ok && dsm_uses > 0) ok = warp_wait_b(&bars.dsm_free, (dsm_uses - 1) & 1, wctx);
@@ -557,12 +587,17 @@ __global__ void __launch_bounds__(BwdWideCfg<HD>::NTHREADS, 1)
           tmem_ld_wait();
           uint32_t dk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = cc * 32 + 2 * e;
-            const float p0f = __uint_as_float(pk[cc][e] << 16);
-            const float p1f = __uint_as_float(pk[cc][e] & 0xFFFF0000u);
-            dk[e] = pack_bf16x2(p0f * (__uint_as_float(sv[2 * e]) - dlt_c[c0]),
-                                p1f * (__uint_as_float(sv[2 * e + 1]) - dlt_c[c0 + 1]));
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 nd = nd4[cc * 8 + q4];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int e = 2 * q4 + hh;
+              const uint64_t t2 = f2_add(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                                         hh == 0 ? f2_pack(nd.x, nd.y) : f2_pack(nd.z, nd.w));
+              float d0, d1;
+              f2_unpack(f2_mul(bf16x2_widen(pk[cc][e]), t2), d0, d1);
+              dk[e] = pack_bf16x2(d0, d1);
+            }
           }
           tmem_st16(tS + 32 + cc * 16, dk);
 #pragma unroll
@@ -654,7 +689,7 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
     if (tr.begin) cudaEventRecord(tr.begin, stream);
     zsa_bwd_pre_kernel<HD><<<int(blocks), 256, 0, stream>>>(
         reinterpret_cast<const __nv_bfloat16*>(a.o), reinterpret_cast<const __nv_bfloat16*>(a.dout),
-        a.delta, a.dq_acc, pairs, a.Hq, twoC);
+        a.lse, a.delta, a.nlse2, a.dq_acc, pairs, a.Hq, twoC);
     cudaError_t e = cudaGetLastError();
     if (tr.end) cudaEventRecord(tr.end, stream);
     if (e != cudaSuccess) return int(e);
@@ -676,16 +711,16 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
     if (!make_map_bf16_sw128(&mk, a.k, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
     if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
-  CUtensorMap mdq;   // the head-major fp32 dQ accumulator, [128 rows][32 d] reduce boxes
-  {
+  CUtensorMap mdq;   // the head-major fp32 dQ accumulator: [32 rows][32 d] reduce boxes
+  {                  // (d <= 128), [64 rows][32 d] (d = 256)
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(rows), uint64_t(a.Hq)};
     const uint64_t strides[2] = {uint64_t(HD) * 4, uint64_t(rows) * HD * 4};
-    const uint32_t box[3] = {32, uint32_t(BQ), 1};
+    const uint32_t box[3] = {32, uint32_t(kWide ? 32 : BQ), 1};
     if (!make_map_f32_sw128(&mdq, a.dq_acc, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
   BwdParams p;
-  p.lse = a.lse;
-  p.delta = a.delta;
+  p.nlse2 = a.nlse2;
+  p.ndelta = a.delta;
   p.dq_acc = a.dq_acc;
   p.dk = reinterpret_cast<__nv_bfloat16*>(a.dk);
   p.dv = reinterpret_cast<__nv_bfloat16*>(a.dv);

@@ -13,8 +13,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kUnitRing = 4;   // claimed units in flight between the producer and the others
 
 struct BwdParams {
-  const float* lse;
-  const float* delta;
+  const float* nlse2;         // -lse * log2(e), [shards][B][Hq][2C] (K2)
+  const float* ndelta;        // -Delta, same layout (K2)
   float* dq_acc;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;

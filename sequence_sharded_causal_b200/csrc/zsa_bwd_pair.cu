@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
             tma_load_3d(smem + Cfg::SMEM_S + st * Cfg::SLOT_BYTES + kb * BQ * 128,
                         rank == 0 ? &map_q : &map_do, &bars.s_full[st], kb * 64, h, row0);
           const int64_t stat = (rb * prm.Hq + h) * twoC + int64_t(w.i) * BQ;
-          bulk_load(smem + Cfg::SMEM_STAT + st * BQ * 4, (rank == 0 ? prm.lse : prm.delta) + stat,
+          bulk_load(smem + Cfg::SMEM_STAT + st * BQ * 4, (rank == 0 ? prm.nlse2 : prm.ndelta) + stat,
                     BQ * 4, &bars.s_full[st]);
           ++s_fills[st];
           ++s_it;
@@ -473,8 +473,8 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = 2 * e;
-            const float x0 = fmaf(__uint_as_float(sv[c0]), prm.scale_log2, -stat_c[c0] * kLog2e);
-            const float x1 = fmaf(__uint_as_float(sv[c0 + 1]), prm.scale_log2, -stat_c[c0 + 1] * kLog2e);
+            const float x0 = fmaf(__uint_as_float(sv[c0]), prm.scale_log2, stat_c[c0]);        // -lse log2 e
+            const float x1 = fmaf(__uint_as_float(sv[c0 + 1]), prm.scale_log2, stat_c[c0 + 1]);
             pk[e] = pack_bf16x2(c0 < nvis_lo ? 0.f : ex2_approx(x0),
                                 c0 + 1 < nvis_lo ? 0.f : ex2_approx(x1));
           }
@@ -502,8 +502,8 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
             for (int t = 0; t < 4; ++t) {
               const int c0 = 8 * m + 2 * t;
               pk[4 * m + t] =
-                  pack_bf16x2(__uint_as_float(pw[t] << 16) * (__uint_as_float(sv[c0]) - stat_c[c0]),
-                              __uint_as_float(pw[t] & 0xFFFF0000u) * (__uint_as_float(sv[c0 + 1]) - stat_c[c0 + 1]));
+                  pack_bf16x2(__uint_as_float(pw[t] << 16) * (__uint_as_float(sv[c0]) + stat_c[c0]),   // -Delta
+                              __uint_as_float(pw[t] & 0xFFFF0000u) * (__uint_as_float(sv[c0 + 1]) + stat_c[c0 + 1]));
             }
           }
         }

@@ -12,8 +12,11 @@
 // Any T; N a multiple of 32; K a multiple of 8: tiles past the edges load zeros (TMA
 // out-of-bounds fill) and the epilogue stores only rows < T and 32-column chunks < N.
 //
-// Kernel: persistent CTAs over 128 x 128 output tiles (tile t -> m block t % MT, n block
-// t / MT: CTAs running together share one column block of W_s in L2).  One TMA warp
+// Kernel: persistent CTAs over 128 x 128 output tiles, rastered in bands of 16 row
+// blocks (m fastest inside a band, then n, then the next band): the tiles running together
+// cover a few row blocks of X and a few column blocks of W_s, so each X row block is read
+// from HBM about once instead of once per column block (an m-fastest order over all of
+// T re-read X for every column block: 12x its size at T = 16384, N = 2048).  One TMA warp
 // streams [128 m][64 k] tiles of X (K-major) and [64 k][128 n] tiles of W_s (two 64-wide
 // n boxes, MN-major) through a 6-stage ring; one thread issues tcgen05.mma (M = N = 128,
 // K = 16) into one of two TMEM accumulators; 4 epilogue warps (thread = output row)
@@ -29,6 +32,16 @@
 
 namespace zsa {
 namespace {
+
+// Output tile t -> (m block, n block): bands of kBand row blocks, m fastest in a band.
+constexpr int32_t kBand = 16;
+__device__ __forceinline__ void tile_mn(int32_t t, int32_t mt, int32_t nt, int32_t& mb, int32_t& nb) {
+  const int32_t band = t / (kBand * nt);
+  const int32_t in = t - band * (kBand * nt);
+  const int32_t rows = mt - band * kBand < kBand ? mt - band * kBand : kBand;  // rows in this band
+  nb = in / rows;
+  mb = band * kBand + (in - nb * rows);
+}
 
 struct GemmCfg {
   static constexpr int BM = 128, BN = 128, BK = 64;
@@ -114,7 +127,9 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
       for (int s = 0; s < Cfg::STAGES; ++s) fills[s] = 0;
       bool ok = true;
       for (int32_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int32_t m0 = (t % prm.mt) * Cfg::BM, n0 = (t / prm.mt) * Cfg::BN;
+        int32_t mb, nb;
+        tile_mn(t, prm.mt, prm.nt, mb, nb);
+        const int32_t m0 = mb * Cfg::BM, n0 = nb * Cfg::BN;
         for (int32_t kb = 0; kb < kblocks; ++kb, ++it) {
           const int st = int(it % Cfg::STAGES);
           if (it >= uint32_t(Cfg::STAGES)) ok = mbar_wait(&bars.empty[st], ((it / Cfg::STAGES) - 1) & 1, wctx);
@@ -175,8 +190,10 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int64_t m = int64_t(t % prm.mt) * Cfg::BM + row;
-      const int64_t n0 = int64_t(t / prm.mt) * Cfg::BN;
+      int32_t mb, nb;
+      tile_mn(t, prm.mt, prm.nt, mb, nb);
+      const int64_t m = int64_t(mb) * Cfg::BM + row;
+      const int64_t n0 = int64_t(nb) * Cfg::BN;
       const bool row_in = m < prm.T;
 #pragma unroll 1
       for (int c = 0; c < Cfg::BN / 32; ++c) {
@@ -203,7 +220,7 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
           __syncwarp();
           if (lane == 0) {
             tma_reduce_add_3d(&seg_maps.m[si], box, int32_t(oc),
-                              int32_t(int64_t(t % prm.mt) * Cfg::BM + warp * 32), 0);
+                              int32_t(int64_t(mb) * Cfg::BM + warp * 32), 0);
             bulk_commit_group();
           }
           ++n_red;

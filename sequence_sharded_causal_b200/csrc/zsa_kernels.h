@@ -42,7 +42,8 @@ struct BwdArgs {
   void* dq;
   void* dk;
   void* dv;
-  float* delta;            // [shards][B][Hq][2C] workspace
+  float* delta;            // [shards][B][Hq][2C] workspace: -Delta (written by K2)
+  float* nlse2;            // [shards][B][Hq][2C] workspace: -lse * log2(e) (written by K2)
   float* dq_acc;           // [Hq][shards*B*2C][d] workspace (head-major)
   int64_t S;
   int32_t B, Hq, Hkv, d, D, causal;

@@ -102,7 +102,8 @@ extern "C" int zsa_attn_bwd_noalloc(const zsa_problem* problem, const void* q, c
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse; a.dout = dout;
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.delta = reinterpret_cast<float*>(base + kNoAllocStatusBytes);
-  a.dq_acc = reinterpret_cast<float*>(base + kNoAllocStatusBytes + align256(stats));
+  a.nlse2 = reinterpret_cast<float*>(base + kNoAllocStatusBytes + align256(stats));
+  a.dq_acc = reinterpret_cast<float*>(base + kNoAllocStatusBytes + 2 * align256(stats));
   a.S = problem->S; a.B = int32_t(problem->B); a.Hq = problem->Hq; a.Hkv = problem->Hkv;
   a.d = problem->d; a.D = problem->D; a.causal = problem->causal;
   a.scale = problem->softmax_scale;
