@@ -52,7 +52,11 @@ DEFAULT_CONFIG = "long"
 # the current kernel at the configuration's full size (dram__bytes_read.sum +
 # dram__bytes_write.sum, a one-pass capture; profiles/dram_traffic_bwd_main.md);
 # configurations without a capture report null.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    ("long", "zsa_bwd_wide_kernel"): 18.58e9 + 9.84e9,
+    ("8b_gqa", "zsa_bwd_wide_kernel"): 1.812251e9 + 0.949273e9,
+    ("wide_gqa", "zsa_bwd_pair_kernel"): 35.44e9 + 21.17e9,
+}
 # Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
 CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
 
