@@ -51,6 +51,11 @@ using namespace bwd;
 // the main kernel's element formulas stored ready to add (P^T = 2^(scale log2(e) S^T +
 // (-lse log2 e)) is one FMA, dS^T = P^T (dP^T + (-Delta)) one add and one multiply), and
 // the zeroed dQ accumulator.
+// A warp takes 32 consecutive (row, head) pairs in the stats order (rb, h, j) -- the
+// order of the fp32 [rows-block][Hq][2C] arrays -- so it reads 32 rows of O and dO (HD*2
+// contiguous bytes each), writes each of the two stats arrays with one 128-byte store,
+// and zeroes a contiguous 32*HD-float block of the accumulator (the pairs tile it, so any
+// order zeroes all of it).  2C is a multiple of 128, so 32 consecutive pairs share (rb, h).
 template <int HD>
 __global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                           const __nv_bfloat16* __restrict__ dout,
@@ -60,19 +65,27 @@ __global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* _
                                                           float* __restrict__ dq_acc,
                                                           int64_t n_pairs, int32_t Hq,
                                                           int64_t twoC) {
-  constexpr int LPP = HD / 8;  // lanes per (row, head) pair, 8 bf16 (16 B) per lane
+  constexpr int LPP = HD / 8;   // lanes per pair, 8 bf16 (16 B) per lane
+  constexpr int PPI = 32 / LPP; // pairs per warp iteration
   const int lane = int(threadIdx.x & 31);
-  const int sub = lane % LPP;
+  const int sub = lane % LPP, grp = lane / LPP;
   const int64_t warp_global = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
   const int64_t n_warps = int64_t(gridDim.x) * blockDim.x / 32;
-  for (int64_t base = warp_global * (32 / LPP); base < n_pairs; base += n_warps * (32 / LPP)) {
-    const int64_t pair = base + lane / LPP;
-    float acc = 0.f;
-    if (pair < n_pairs) {
-      const uint4 a = reinterpret_cast<const uint4*>(o + pair * HD)[sub];
-      const uint4 b = reinterpret_cast<const uint4*>(dout + pair * HD)[sub];
+  for (int64_t base = warp_global * 32; base < n_pairs; base += n_warps * 32) {
+    const int64_t rbh = base / twoC;
+    const int64_t j0 = base - rbh * twoC;
+    const int64_t rb = rbh / Hq;
+    const int64_t h = rbh - rb * Hq;
+    float mine = 0.f;                         // lane l ends with pair base + l's rowsum
+#pragma unroll 4
+    for (int it = 0; it < 32 / PPI; ++it) {
+      const int pi = it * PPI + grp;
+      const int64_t el = ((rb * twoC + j0 + pi) * Hq + h) * HD;   // (row, h) in O's layout
+      const uint4 a = reinterpret_cast<const uint4*>(o + el)[sub];
+      const uint4 b = reinterpret_cast<const uint4*>(dout + el)[sub];
       const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
       const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+      float acc = 0.f;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const float2 x = __bfloat1622float2(a2[t]);
@@ -80,22 +93,16 @@ __global__ void __launch_bounds__(256) zsa_bwd_pre_kernel(const __nv_bfloat16* _
         acc = fmaf(x.x, y.x, acc);
         acc = fmaf(x.y, y.y, acc);
       }
-      // zero d floats per (row, head) pair: the pairs tile the whole accumulator, so this
-      // holds for its head-major layout too
-      float4* z = reinterpret_cast<float4*>(dq_acc + pair * HD) + 2 * sub;
+#pragma unroll
+      for (int off = LPP / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const float v = __shfl_sync(0xffffffffu, acc, (lane % PPI) * LPP);
+      if (lane / PPI == it) mine = v;
+      float4* z = reinterpret_cast<float4*>(dq_acc + (base + pi) * HD) + 2 * sub;
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-#pragma unroll
-    for (int off = LPP / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (pair < n_pairs && sub == 0) {
-      const int64_t row = pair / Hq;           // (r*B + b)*2C + j
-      const int32_t h = int32_t(pair % Hq);
-      const int64_t rb = row / twoC, j = row % twoC;
-      const int64_t sidx = (rb * Hq + h) * twoC + j;
-      ndelta[sidx] = -acc;
-      nlse2[sidx] = -lse[sidx] * kLog2e;
-    }
+    ndelta[base + lane] = -mine;
+    nlse2[base + lane] = -lse[base + lane] * kLog2e;
   }
 }
 
@@ -681,7 +688,7 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
   // K2: Delta and a zeroed dQ accumulator
   {
     const int64_t pairs = rows * a.Hq;
-    const int64_t warps_needed = (pairs + (256 / HD) * 4 - 1) / ((256 / HD) * 4);
+    const int64_t warps_needed = (pairs + 31) / 32;
     int64_t blocks = (warps_needed + 7) / 8;
     if (blocks > int64_t(sms) * 16) blocks = int64_t(sms) * 16;
     if (blocks < 1) blocks = 1;
@@ -712,10 +719,10 @@ int launch_bwd_hd(const BwdArgs& a, cudaStream_t stream) {
     if (!make_map_bf16_sw128(&mv, a.v, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
   CUtensorMap mdq;   // the head-major fp32 dQ accumulator: [32 rows][32 d] reduce boxes
-  {                  // (d <= 128), [64 rows][32 d] (d = 256)
+  {
     const uint64_t dims[3] = {uint64_t(HD), uint64_t(rows), uint64_t(a.Hq)};
     const uint64_t strides[2] = {uint64_t(HD) * 4, uint64_t(rows) * HD * 4};
-    const uint32_t box[3] = {32, uint32_t(kWide ? 32 : BQ), 1};
+    const uint32_t box[3] = {32, 32, 1};
     if (!make_map_f32_sw128(&mdq, a.dq_acc, 3, dims, strides, box)) return int(cudaErrorInvalidValue);
   }
   BwdParams p;

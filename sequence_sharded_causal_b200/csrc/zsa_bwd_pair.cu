@@ -360,9 +360,10 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
   } else if (warp >= Cfg::WARP_DQ) {
     // ------------------------------------------------------------ dQ warps (CTA 0)
     // Each dQ^T half of a slot (TMEM lane = d within the half, column = q row) is staged
-    // as four [64 q][32 d] fp32 boxes (one per warp, 128-byte rows, 128-byte swizzle) in
-    // the staging buffer and reduced into the accumulator by one TMA bulk reduce-add per
-    // warp; the second half reuses the box after the first half's reduce has read it.
+    // as [32 q][32 d] fp32 boxes (128-byte rows, 128-byte swizzle) in a ring of two per
+    // warp in the staging buffer, each reduced into the accumulator by one TMA bulk
+    // reduce-add: a box is rewritten once the reduce issued two boxes earlier has read
+    // it, so staging overlaps the reduces instead of waiting for each to drain.
     if (rank == 0) {
       const int qw = warp - Cfg::WARP_DQ;
       const uint32_t tXT = tmem + Cfg::TM_XT + (uint32_t(qw * 32) << 16);
@@ -396,19 +397,23 @@ __global__ void __launch_bounds__(PairCfg::NTHREADS, 1)
             if (lane == 0) mbar_arrive(&bars.dq_empty[hh]);
             const uint32_t within = uint32_t(lane & 3) * 4;
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+            for (int t = 0; t < 2; ++t) {
+              // [32 q][32 d] boxes in a ring of two per warp: the box written now was last
+              // used two reduces ago, which must have read it (at most one in flight)
+              uint8_t* bx = box + ((hh * 2 + t) & 1) * (32 * 128);
+              if (lane == 0) bulk_wait_group_read1();
+              __syncwarp();
 #pragma unroll
               for (int c = 0; c < 32; ++c)
-                *reinterpret_cast<uint32_t*>(box + sw128_offset(uint32_t(t * 32 + c), uint32_t(lane >> 2)) +
-                                             within) = v[t][c];
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_reduce_add_3d(&map_dq, box, hh * 128 + qw * 32, row0, h);
-              bulk_commit_group();
-              bulk_wait_group_read0();       // the box may be overwritten
+                *reinterpret_cast<uint32_t*>(bx + sw128_offset(uint32_t(c), uint32_t(lane >> 2)) + within) =
+                    v[t][c];
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_reduce_add_3d(&map_dq, bx, hh * 128 + qw * 32, row0 + t * 32, h);
+                bulk_commit_group();
+              }
             }
-            __syncwarp();
           }
           dq_ph ^= 1;
         }
