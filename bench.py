@@ -55,7 +55,7 @@ DEFAULT_CONFIG = "long"
 MEASURED_TRAFFIC = {
     ("long", "zsa_bwd_wide_kernel"): 18.58e9 + 9.84e9,
     ("8b_gqa", "zsa_bwd_wide_kernel"): 1.812251e9 + 0.949273e9,
-    ("wide_gqa", "zsa_bwd_pair_kernel"): 35.44e9 + 21.17e9,
+    ("wide_gqa", "zsa_bwd_pair_kernel"): 35.15e9 + 20.32e9,
 }
 # Oracle sample: full fwd+bwd at a reduced sequence length (same B, heads, d, D).
 CPU_SAMPLE_S = {"tiny": 256, "7b_mha": 1024, "8b_gqa": 1024, "wide_gqa": 512, "long": 2048}
