@@ -43,11 +43,15 @@ __device__ __forceinline__ void tile_mn(int32_t t, int32_t mt, int32_t nt, int32
   mb = band * kBand + (in - nb * rows);
 }
 
+// Tiles of 128 x TBN outputs: TBN = 256 (N = 256 MMAs) halves the operand bytes staged per
+// FLOP against TBN = 128 (every 128 rows of X feed twice the columns), for GEMMs with
+// enough tiles; TBN = 128 keeps small-N steps (a few tiles per SM) from wasting columns.
+template <int TBN>
 struct GemmCfg {
-  static constexpr int BM = 128, BN = 128, BK = 64;
-  static constexpr int STAGES = 6;
+  static constexpr int BM = 128, BN = TBN, BK = 64;
+  static constexpr int STAGES = TBN == 256 ? 4 : 6;
   static constexpr int A_BYTES = BM * BK * 2;     // 16 KB
-  static constexpr int B_BYTES = BK * BN * 2;     // 16 KB: [2 n blocks][64 k][128 B]
+  static constexpr int B_BYTES = BK * BN * 2;     // [BN / 64 n blocks][64 k][128 B]
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STG_BYTES = 4 * 2 * 32 * 128;   // 4 warps x 2 boxes of [32 rows][32 fp32]
   static constexpr int SMEM_STG = STAGES * STAGE_BYTES;
@@ -55,7 +59,7 @@ struct GemmCfg {
   static constexpr int WARP_LOAD = 4;
   static constexpr int WARP_MMA = 5;
   static constexpr int NTHREADS = 6 * 32;
-  static constexpr uint32_t TM_COLS = 256;        // two 128-column accumulators
+  static constexpr uint32_t TM_COLS = 2 * BN;     // two BN-column accumulators
   static_assert(SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 };
 
@@ -74,16 +78,17 @@ struct GemmParams {
 };
 
 struct GemmBars {
-  uint64_t full[GemmCfg::STAGES], empty[GemmCfg::STAGES];
+  uint64_t full[6], empty[6];                      // GemmCfg<BN>::STAGES <= 6
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;
 };
 
-__global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
+template <int TBN>
+__global__ void __launch_bounds__(GemmCfg<TBN>::NTHREADS, 1)
     zsa_proj_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                          const __grid_constant__ CUtensorMap map_w,
                          const __grid_constant__ SegMaps seg_maps, const GemmParams prm) {
-  using Cfg = GemmCfg;
+  using Cfg = GemmCfg<TBN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -137,7 +142,7 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
           uint8_t* sa = smem + st * Cfg::STAGE_BYTES;
           mbar_expect_tx(&bars.full[st], Cfg::STAGE_BYTES);
           tma_load_3d(sa, &map_x, &bars.full[st], kb * Cfg::BK, m0, 0);
-          for (int nb = 0; nb < 2; ++nb)
+          for (int nb = 0; nb < Cfg::BN / 64; ++nb)
             tma_load_3d(sa + Cfg::A_BYTES + nb * (Cfg::BK * 128), &map_w, &bars.full[st],
                         n0 + nb * 64, kb * Cfg::BK, 0);
           ++fills[st];
@@ -247,10 +252,9 @@ __global__ void __launch_bounds__(GemmCfg::NTHREADS, 1)
   if (warp == Cfg::WARP_MMA) tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
-}  // namespace
-
-int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
-  using Cfg = GemmCfg;
+template <int TBN>
+int launch_proj_gemm_bn(const ProjArgs& a, cudaStream_t stream) {
+  using Cfg = GemmCfg<TBN>;
   CUtensorMap mx, mw;
   {
     const uint64_t dims[3] = {uint64_t(a.K), uint64_t(a.T), 1};
@@ -283,7 +287,7 @@ int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
   const int smem = Cfg::SMEM_BYTES + 1024;
-  int e = ensure_smem_attr(reinterpret_cast<const void*>(zsa_proj_gemm_kernel), smem);
+  int e = ensure_smem_attr(reinterpret_cast<const void*>(zsa_proj_gemm_kernel<TBN>), smem);
   if (e != int(cudaSuccess)) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -293,10 +297,23 @@ int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
   if (grid <= 0) return int(cudaSuccess);
   const TraceEvents tr = trace_events(5);
   if (tr.begin) cudaEventRecord(tr.begin, stream);
-  zsa_proj_gemm_kernel<<<grid, Cfg::NTHREADS, smem, stream>>>(mx, mw, sm, p);
+  zsa_proj_gemm_kernel<TBN><<<grid, Cfg::NTHREADS, smem, stream>>>(mx, mw, sm, p);
   const cudaError_t err = cudaGetLastError();
   if (tr.end) cudaEventRecord(tr.end, stream);
   return int(err);
+}
+
+}  // namespace
+
+// 256-wide tiles when N divides into them and they still give every SM at least two
+// tiles; 128-wide otherwise.
+int launch_proj_gemm(const ProjArgs& a, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles256 = ((a.T + 127) / 128) * (a.N / 256);
+  if (a.N % 256 == 0 && tiles256 >= 2 * int64_t(sms)) return launch_proj_gemm_bn<256>(a, stream);
+  return launch_proj_gemm_bn<128>(a, stream);
 }
 
 }  // namespace zsa

@@ -37,7 +37,9 @@ def _rand(shape, seed, scale=1.0):
 
 @pytest.mark.parametrize("T,K,N", [(128, 64, 128), (256, 512, 384), (1024, 4096, 768),
                                    (384, 1280, 1024),
-                                   (200, 72, 160)])    # ragged: T, N, K past the tile edges
+                                   (200, 72, 160),     # ragged: T, N, K past the tile edges
+                                   (4096, 512, 2560),  # 128 x 256 tiles (N = 256 MMAs)
+                                   (4000, 264, 2560)]) # 128 x 256 tiles, ragged T and K
 def test_project_bf16_matches_oracle(oracle, T, K, N):
     x, w = _rand((T, K), 1), _rand((K, N), 2, 0.05)
     ws = torch.empty(256, dtype=torch.uint8, device="cuda")
@@ -66,6 +68,22 @@ def test_project_segments_and_fp32_accumulate(oracle):
     assert torch.count_nonzero(a[:, :40]).item() == 0 and torch.count_nonzero(a[:, 136:]).item() == 0
     check_bf16(b.float().cpu().numpy(), ref2[:, 96:256])
     ref_acc = oracle.project(x1, w)[:, 256:] + ref2[:, 256:]
+    rms = float(np.sqrt((ref_acc ** 2).mean()))
+    assert float(np.abs(acc.cpu().numpy() - ref_acc).max()) <= 1e-4 * rms
+
+
+def test_project_wide_tiles_fp32_accumulate(oracle):
+    # enough 128 x 256 tiles for the wide-tile build: a bf16 segment and an fp32 one
+    T, K, N = 4096, 256, 2560
+    x, w = _rand((T, K), 6), _rand((K, N), 7, 0.05)
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    a = torch.zeros(T, 512, dtype=torch.bfloat16, device="cuda")
+    acc = torch.full((T, 2048), 1.0, dtype=torch.float32, device="cuda")
+    zsa.zsa_tsp_project(x.cuda(), w.cuda(), [(a, 512, 512, 0), (acc, 2048, 2048, 1)], ws)
+    assert zsa.zsa_device_status(ws) == zsa.ZSA_OK
+    ref = oracle.project(x, w)
+    check_bf16(a.float().cpu().numpy(), ref[:, :512])
+    ref_acc = ref[:, 512:] + 1.0
     rms = float(np.sqrt((ref_acc ** 2).mean()))
     assert float(np.abs(acc.cpu().numpy() - ref_acc).max()) <= 1e-4 * rms
 
