@@ -230,19 +230,28 @@ def run_zsa(args, c, name):
     stream = torch.cuda.current_stream(dev)
     if world == 1:
         # one launch over all D shards, natural-order K/V (the gathered buffer)
-        o = torch.empty_like(q)
-        lse = torch.empty(D, B, Hq, S // D, dtype=torch.float32, device=dev)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         ws_f = torch.empty(zsa.zsa_workspace_bytes(problem, 0), dtype=torch.uint8, device=dev)
         ws_b = torch.empty(zsa.zsa_workspace_bytes(problem, 1), dtype=torch.uint8, device=dev)
 
-        def step():
-            zsa.zsa_attn_fwd(problem, q, k, v, o, lse, ws_f, stream=stream)
-            zsa.zsa_attn_bwd(problem, q, k, v, o, lse, do, dq, dk, dv, ws_b, stream=stream)
+        def make_set(q, k, v, do):
+            """A step over one set of device buffers: (inputs, outputs, step)."""
+            o = torch.empty_like(q)
+            lse = torch.empty(D, B, Hq, S // D, dtype=torch.float32, device=dev)
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+            def run():
+                zsa.zsa_attn_fwd(problem, q, k, v, o, lse, ws_f, stream=stream)
+                zsa.zsa_attn_bwd(problem, q, k, v, o, lse, do, dq, dk, dv, ws_b, stream=stream)
+            return (q, k, v, do), (o, lse, dq, dk, dv), run
+
+        inputs_t, outputs_t, step = make_set(q, k, v, do)
+        o = outputs_t[0]
+
+        def second_set():
+            return make_set(*(torch.empty_like(x) for x in inputs_t))
 
         def device_status():
             return zsa.zsa_device_status(ws_f) or zsa.zsa_device_status(ws_b)
-        inputs_t, outputs_t = (q, k, v, do), (o, lse, dq, dk, dv)
     else:
         from sequence_sharded_causal_b200 import dist as zdist
         core = zdist.ShardedAttention(B, S, Hq, Hkv, d, D, rank, world, device=dev)
@@ -263,6 +272,7 @@ def run_zsa(args, c, name):
         def device_status():
             return core.status()
         inputs_t, outputs_t = (q, k, v, do), (o, lse, dq, dk, dv)
+        second_set = None      # lse lives in the core: one buffer set, copies not overlapped
 
     def barrier():
         if dist is not None:
@@ -323,20 +333,47 @@ def run_zsa(args, c, name):
     bi = sum(x.numel() * x.element_size() for x in h_in)
     bo = sum(x.numel() * x.element_size() for x in h_out)
     K2 = max(1, min(K, 10))
+    # One GPU: two sets of device buffers and two copy streams, so step i+1's inputs go
+    # up and step i-1's results come down while step i's kernels run (a set is reused
+    # only after its previous step's kernels and read-back are done).  Several ranks:
+    # one set (the core owns lse), copies in line with the kernels.
+    sets = [(inputs_t, outputs_t, step)]
+    if second_set is not None:
+        sets.append(second_set())
+    e2e_mode = ("double-buffered device sets; H2D of step i+1 and D2H of step i-1 on two "
+                "copy streams overlap step i" if len(sets) == 2 else "serial: H2D, step, D2H")
+    h2d_s = torch.cuda.Stream(dev)
+    d2h_s = torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_done, ev_out = [ev() for _ in range(K2)], [ev() for _ in range(K2)], [ev() for _ in range(K2)]
     barrier()
     torch.cuda.synchronize(dev)
-    t0 = time.perf_counter()
     x0 = torch.cuda.Event(enable_timing=True)
     x1 = torch.cuda.Event(enable_timing=True)
     x0.record(stream)
-    for _ in range(K2):
-        for dst, src in zip(inputs_t, h_in):
-            dst.copy_(src, non_blocking=True)
-        step()
-        for dst, src in zip(h_out, outputs_t):
-            dst.copy_(src, non_blocking=True)
+    for i in range(K2):
+        ins, outs, run = sets[i % len(sets)]
+        h2d_s.wait_event(x0)
+        if i >= len(sets):
+            h2d_s.wait_event(ev_done[i - len(sets)])     # the set's last step has read it
+        with torch.cuda.stream(h2d_s):
+            for dst, src in zip(ins, h_in):
+                dst.copy_(src, non_blocking=True)
+        ev_in[i].record(h2d_s)
+        stream.wait_event(ev_in[i])
+        if i >= len(sets):
+            stream.wait_event(ev_out[i - len(sets)])     # its results have been read back
+        run()
+        ev_done[i].record(stream)
+        d2h_s.wait_event(ev_done[i])
+        with torch.cuda.stream(d2h_s):
+            for dst, src in zip(h_out, outs):
+                dst.copy_(src, non_blocking=True)
+        ev_out[i].record(d2h_s)
+    stream.wait_event(ev_out[K2 - 1])
     x1.record(stream)
     torch.cuda.synchronize(dev)
+    del sets
     e2e_ms = x0.elapsed_time(x1) / K2
     e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist is not None:
@@ -392,7 +429,7 @@ def run_zsa(args, c, name):
                      "frac_of_sustained": (dom_tf / peak_sus) if peak_sus else None,
                      "traffic": traffic},
         "e2e": {"value": job_tflops((ff + bf) / world, world, e2e_ms), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo},
+                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "mode": e2e_mode},
         "hbm_kernels": hbm_kernels,
         "gpu_launches": 4 * K,
         "clocks": clk,
