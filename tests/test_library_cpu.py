@@ -106,6 +106,26 @@ def test_argument_errors(L):
     assert (t.block_q, t.block_k, t.slots) == (128, 128, 2)
 
 
+def test_size_limits(L):
+    # key-tile counts are packed in 16 bits: S / 128 must stay below 65536
+    assert _rc_fwd(L, zsa.make_problem(1, 65536 * 128, 4, 2, 128, 1)) == zsa.ZSA_ERR_SHAPE
+    assert _rc_fwd(L, zsa.make_problem(1, 65535 * 128, 4, 2, 128, 1), ws_bytes=64) == zsa.ZSA_ERR_WORKSPACE
+    # B * S < 2^31: TMA row coordinates are int32
+    assert _rc_fwd(L, zsa.make_problem(2 ** 15, 2 ** 16, 4, 2, 128, 2)) == zsa.ZSA_ERR_SHAPE
+    assert _rc_fwd(L, zsa.make_problem(2 ** 14, 2 ** 16, 4, 2, 128, 2), ws_bytes=64) == zsa.ZSA_ERR_WORKSPACE
+    # the merge indexes rows * Hq * d in 32 bits
+    big = zsa.make_problem(1, 2 ** 20, 32, 8, 128, 16)          # 2^20 * 32 * 128 = 2^32
+    parts = (ctypes.c_void_p * 2)(16, 16)
+    lses = (ctypes.c_void_p * 2)(16, 16)
+    assert L.zsa_attn_merge(ctypes.byref(big), 2, parts, lses, 16, 16, None) == zsa.ZSA_ERR_SHAPE
+    ok = zsa.make_problem(1, 2 ** 18, 32, 8, 128, 16)            # 2^30: below the limit
+    assert L.zsa_attn_merge(ctypes.byref(ok), 2, parts, lses, 16, 16, None) not in (
+        zsa.ZSA_ERR_SHAPE, zsa.ZSA_ERR_INVALID)
+    assert L.zsa_attn_merge(ctypes.byref(ok), 0, parts, lses, 16, 16, None) == zsa.ZSA_ERR_INVALID
+    assert L.zsa_attn_merge(ctypes.byref(ok), zsa.ZSA_MERGE_MAX_PARTS + 1, parts, lses, 16, 16,
+                            None) == zsa.ZSA_ERR_INVALID
+
+
 def test_permute_argument_errors(L):
     good = zsa.make_problem(2, 1024, 4, 2, 128, 2)
     P = ctypes.byref(good)
