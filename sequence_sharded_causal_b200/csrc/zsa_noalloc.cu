@@ -1,7 +1,7 @@
 // zsa_noalloc.cu -- the backward pass for callers that cannot allocate device memory.
 //
-// zsa_attn_bwd needs a caller-provided workspace (status word, Delta, fp32 dQ
-// accumulator).  Some callers have no way to provide one at the call site: plugins
+// zsa_attn_bwd needs a caller-provided workspace (status word, -Delta, -lse*log2(e), fp32
+// dQ accumulator).  Some callers have no way to provide one at the call site: plugins
 // inside a host runtime whose device memory is entirely owned and pre-planned by that
 // runtime (they may not call cudaMalloc, and the runtime offers no scratch hook), or a
 // C caller that links the library without any allocator of its own.
