@@ -280,9 +280,8 @@ ZSA_API int zsa_tsp_project(int64_t T, int64_t K, int64_t N, const void* x, int6
  * or C callers without an allocator of their own.  Arguments and results are those of
  * zsa_attn_bwd; the scratch (status word, -Delta, -lse*log2(e), fp32 dQ accumulator) is
  * a fixed static device array of ZSA_NOALLOC_SCRATCH_BYTES, resident until the process
- * exits on every
- * GPU on which the library's module is loaded (under CUDA's eager module loading, every
- * GPU the process has a context on).
+ * exits on every GPU on which the library's module is loaded (under CUDA's eager module
+ * loading, every GPU the process has a context on).
  *  - Problems needing more scratch than that (zsa_workspace_bytes(problem, 1) >
  *    ZSA_NOALLOC_SCRATCH_BYTES) return ZSA_ERR_WORKSPACE before anything is enqueued.
  *  - All calls on a device share the array and it keeps the last call's contents:
