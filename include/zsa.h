@@ -161,7 +161,10 @@ ZSA_API int zsa_attn_fwd(const zsa_problem* problem, const void* q, const void* 
                  void* o, float* lse, void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /* Backward: dq (Q layout), dk, dv (K layout), all bf16, overwritten (not accumulated).
- * o and lse must come from zsa_attn_fwd on the same inputs.
+ * o and lse must come from zsa_attn_fwd on the same inputs.  dk and dv are the same on
+ * every run; dq sums the key tiles' contributions with fp32 reduce-adds whose order
+ * between thread blocks is not fixed, so runs may differ by that fp32 rounding (seen
+ * through the bf16 output).
  * Defined by: the pages describe only the forward; this is the exact gradient of
  * <dO, O> for the forward above (the reading taken where the pages are silent), with
  * dK/dV summed over every shard as the reduce-scatter back to the owning shards of the

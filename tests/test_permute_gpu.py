@@ -64,3 +64,40 @@ def test_permute_shard_range(oracle):
         mask[pos] = True
         assert torch.equal(got[:, torch.from_numpy(mask)], x[:, torch.from_numpy(mask)])
         assert (got[:, torch.from_numpy(~mask)] == 7.0).all()
+
+
+def test_permuted_inputs_drive_the_attention(oracle):
+    # Q and K/V brought to shard-major order by K5 feed the attention kernels directly:
+    # the same values reach the same tiles in the same order as with the generator's own
+    # layout and natural-order K/V, so the results are identical
+    B, S, Hq, Hkv, d, D = 1, 2048, 4, 2, 128, 4
+    from sequence_sharded_causal_b200 import inputs
+    q_nat, k, v, _, _ = inputs.make_inputs(B, S, Hq, Hkv, d, 11)
+    perm, _ = oracle.partition(S, D)
+    q_ref = inputs.to_shard_major(q_nat, perm, D).cuda()
+    kc, vc = k.cuda(), v.cuda()
+    q_k5 = zsa.to_shard_major(q_nat.cuda(), D)
+    assert torch.equal(q_k5, q_ref)
+    o_ref, l_ref = zsa.attn_fwd(q_ref, kc, vc, D)
+    k_sm, v_sm = zsa.to_shard_major(kc, D), zsa.to_shard_major(vc, D)
+    o_sm, l_sm = zsa.attn_fwd(q_k5, k_sm, v_sm, D, kv_layout=zsa.ZSA_KV_SHARD_MAJOR)
+    torch.cuda.synchronize()
+    assert torch.equal(o_sm, o_ref) and torch.equal(l_sm, l_ref)
+    # and back: O in position order
+    o_nat = zsa.from_shard_major(o_sm, D)
+    torch.cuda.synchronize()
+    assert torch.equal(o_nat.cpu(), inputs.from_shard_major(o_ref.cpu(), perm))
+    # the backward with shard-major K/V writes dK / dV in that order; K5 brings them back
+    _, _, _, do_nat, _ = inputs.make_inputs(B, S, Hq, Hkv, d, 11)
+    do = zsa.to_shard_major(do_nat.cuda(), D)
+    dq_ref, dk_ref, dv_ref = zsa.attn_bwd(q_ref, kc, vc, o_ref, l_ref, do, D)
+    dq_sm, dk_sm, dv_sm = zsa.attn_bwd(q_k5, k_sm, v_sm, o_sm, l_sm, do, D,
+                                       kv_layout=zsa.ZSA_KV_SHARD_MAJOR)
+    torch.cuda.synchronize()
+    # dK / dV are accumulated inside one CTA per key tile: identical.  dQ sums the key
+    # tiles' contributions with fp32 reduce-adds whose order between CTAs is not fixed,
+    # so two runs agree to fp32 summation-order rounding before the bf16 rounding
+    assert torch.equal(zsa.from_shard_major(dk_sm, D), dk_ref)
+    assert torch.equal(zsa.from_shard_major(dv_sm, D), dv_ref)
+    diff = (dq_sm.float() - dq_ref.float()).norm() / dq_ref.float().norm()
+    assert float(diff) < 1e-3, float(diff)
