@@ -29,6 +29,12 @@
 // as P_s(n) is published (p_full), by the other issuing thread, so neither list waits
 // behind the other.  The softmax waits for PV_s(n-1) (pv_done) only before it
 // overwrites P_s or rescales O_s, after its exponentials.
+//
+// The key-block build (KR = true, zsa_attn_fwd_block) is the same kernel restricted to the
+// keys of one K/V block, the partial of a ring-attention step ("AutoSP" summary, sections
+// 1 and 4): each slot's key tiles are clamped to the block's, K/V rows come from the
+// block's linear row map, the mask adds the block's bounds, and a row that sees no key of
+// the block ends as O = 0, lse = -inf.
 #include <cuda_bf16.h>
 
 #include <cmath>
