@@ -12,15 +12,16 @@
 // Any T; N a multiple of 32; K a multiple of 8: tiles past the edges load zeros (TMA
 // out-of-bounds fill) and the epilogue stores only rows < T and 32-column chunks < N.
 //
-// Kernel: persistent CTAs over 128 x 128 output tiles, rastered in bands of 16 row
-// blocks (m fastest inside a band, then n, then the next band): the tiles running together
-// cover a few row blocks of X and a few column blocks of W_s, so each X row block is read
-// from HBM about once instead of once per column block (an m-fastest order over all of
-// T re-read X for every column block: 12x its size at T = 16384, N = 2048).  One TMA warp
-// streams [128 m][64 k] tiles of X (K-major) and [64 k][128 n] tiles of W_s (two 64-wide
-// n boxes, MN-major) through a 6-stage ring; one thread issues tcgen05.mma (M = N = 128,
-// K = 16) into one of two TMEM accumulators; 4 epilogue warps (thread = output row)
-// drain the other accumulator meanwhile.  fp32-accumulate chunks leave by TMA bulk
+// Kernel: persistent CTAs over 128 x BN output tiles (BN = 256 where N and the tile
+// count allow, else 128), rastered in bands of 16 row blocks (m fastest inside a band,
+// then n, then the next band): the tiles running together cover a few row blocks of X and
+// a few column blocks of W_s, so each X row block is read from HBM about once instead of
+// once per column block (an m-fastest order over all of T re-read X for every column
+// block: 12x its size at T = 16384, N = 2048).  One TMA warp streams [128 m][64 k] tiles
+// of X (K-major) and [64 k][BN n] tiles of W_s (64-wide n boxes, MN-major) through a ring
+// of 4 (BN = 256) or 6 stages; one thread issues tcgen05.mma (M = 128, N = BN, K = 16)
+// into one of two TMEM accumulators; 4 epilogue warps (thread = output row) drain the
+// other accumulator meanwhile.  fp32-accumulate chunks leave by TMA bulk
 // reduce-add (each warp stages its [32 rows][32 columns] in a double-buffered,
 // 128B-swizzled box), so the accumulator is never read back by the SM; bf16 chunks are
 // stored directly.  Every wait is bounded.
